@@ -1,0 +1,15 @@
+"""B200-native attention forward + JVP (the rCM / sCM hot path).
+
+``attn_jvp_fwd`` returns O = softmax(s Q K^T) V, its tangent O' along
+(Q', K', V') and the row log-sum-exp, computed by hand-written sm_100a
+kernels behind a small C ABI (``include/attn_jvp.h``).  Importing this package
+does not load the CUDA library; the first call does, and fails loudly if it
+has not been built.
+"""
+from .api import (ATTN_JVP_ERR_ALIGN, ATTN_JVP_ERR_HEADDIM, ATTN_JVP_ERR_LAUNCH,  # noqa: F401
+                  ATTN_JVP_ERR_NULL, ATTN_JVP_ERR_SHAPE, ATTN_JVP_ERR_TIMEOUT,
+                  ATTN_JVP_ERR_VALUE, ATTN_JVP_OK, AttnJvpError, attn_jvp_check,
+                  attn_jvp_fwd, attn_jvp_status_string, library_path)
+
+__all__ = ["attn_jvp_fwd", "attn_jvp_check", "attn_jvp_status_string", "AttnJvpError",
+           "library_path"]

@@ -1,0 +1,155 @@
+"""Python binding of the C ABI in ``include/attn_jvp.h``.
+
+Argument marshalling only: torch supplies device memory and the stream, the
+library does all of the work.  There is no CPU or library fallback; if the
+CUDA library is missing the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+from .build import LIB_PATH
+
+ATTN_JVP_OK = 0
+ATTN_JVP_ERR_NULL = -1
+ATTN_JVP_ERR_SHAPE = -2
+ATTN_JVP_ERR_HEADDIM = -3
+ATTN_JVP_ERR_ALIGN = -4
+ATTN_JVP_ERR_LAUNCH = -5
+ATTN_JVP_ERR_TIMEOUT = -6
+ATTN_JVP_ERR_VALUE = -7
+ATTN_JVP_DEBUG_STARVE_Q = 1
+
+EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_debug", "attn_jvp_check", "attn_jvp_status_string",
+            "attn_jvp_version")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class AttnJvpError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = attn_jvp_status_string(status)
+        super().__init__(f"{what}: {msg} (status {status})" if what else f"{msg} (status {status})")
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def load_library():
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"CUDA library {LIB_PATH} is not built; run "
+                    "`python -m attention_jvp_fwd_b200.build` (nvcc, sm_100a)")
+            lib = ctypes.CDLL(LIB_PATH)
+            vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+            lib.attn_jvp_fwd.restype = i32
+            lib.attn_jvp_fwd.argtypes = [vp] * 9 + [i32] * 5 + [f32, vp, vp]
+            lib.attn_jvp_fwd_debug.restype = i32
+            lib.attn_jvp_fwd_debug.argtypes = [vp] * 9 + [i32] * 5 + [f32, vp, vp,
+                                                                     ctypes.c_uint64, i32]
+            lib.attn_jvp_check.restype = i32
+            lib.attn_jvp_check.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+            lib.attn_jvp_status_string.restype = ctypes.c_char_p
+            lib.attn_jvp_status_string.argtypes = [i32]
+            lib.attn_jvp_version.restype = i32
+            lib.attn_jvp_version.argtypes = []
+            _lib = lib
+    return _lib
+
+
+def attn_jvp_status_string(status: int) -> str:
+    return load_library().attn_jvp_status_string(int(status)).decode()
+
+
+def _check_inputs(q, k, v, q_dot, k_dot, v_dot):
+    for name, t in (("q", q), ("k", k), ("v", v), ("q_dot", q_dot), ("k_dot", k_dot),
+                    ("v_dot", v_dot)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [B, H, L, d]")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be 4-D [B, H, L, d]")
+        if t.device != q.device:
+            raise ValueError("all tensors must be on one device")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    for name, t, L in (("k", k, Lk), ("v", v, Lk), ("q_dot", q_dot, Lq), ("k_dot", k_dot, Lk),
+                       ("v_dot", v_dot, Lk)):
+        if tuple(t.shape) != (B, H, L, d):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {(B, H, L, d)}")
+    return B, H, Lq, Lk, d
+
+
+def _stream_handle(device, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(int(stream.cuda_stream))
+
+
+def attn_jvp_fwd(q, k, v, q_dot, k_dot, v_dot, scale: float | None = None, kv_len=None,
+                 out=None, stream=None, *, _debug_timeout_ns: int | None = None,
+                 _debug_flags: int = 0):
+    """O = softmax(scale Q K^T) V, its tangent O' along (Q', K', V'), and lse.
+
+    q, q_dot: bf16 [B, H, Lq, d]; k, v, k_dot, v_dot: bf16 [B, H, Lk, d];
+    d in {64, 128}; kv_len: optional int32 [B] on the same device (keys
+    j >= kv_len[b] are masked).  scale defaults to 1/sqrt(d).  ``out`` may
+    supply (o, o_dot, lse) buffers.  Queued on ``stream`` (default: the
+    current stream).  Returns (o, o_dot, lse) with lse fp32 [B, H, Lq].
+    """
+    B, H, Lq, Lk, d = _check_inputs(q, k, v, q_dot, k_dot, v_dot)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    kv_ptr = None
+    if kv_len is not None:
+        if (not isinstance(kv_len, torch.Tensor) or kv_len.dtype != torch.int32
+                or kv_len.device != q.device or tuple(kv_len.shape) != (B,)
+                or not kv_len.is_contiguous()):
+            raise ValueError("kv_len must be a contiguous int32 [B] tensor on q's device")
+        kv_ptr = kv_len.data_ptr()
+    if out is None:
+        o = torch.empty_like(q)
+        od = torch.empty_like(q)
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    else:
+        o, od, lse = out
+    lib = load_library()
+    ptrs = [t.data_ptr() for t in (q, k, v, q_dot, k_dot, v_dot, o, od, lse)]
+    sh = _stream_handle(q.device, stream)
+    with torch.cuda.device(q.device):
+        if _debug_timeout_ns is None and not _debug_flags:
+            rc = lib.attn_jvp_fwd(*ptrs, B, H, Lq, Lk, d, float(scale), kv_ptr, sh)
+        else:
+            rc = lib.attn_jvp_fwd_debug(*ptrs, B, H, Lq, Lk, d, float(scale), kv_ptr, sh,
+                                        int(_debug_timeout_ns or 0), int(_debug_flags))
+    if rc != ATTN_JVP_OK:
+        raise AttnJvpError(rc, "attn_jvp_fwd")
+    return o, od, lse
+
+
+def attn_jvp_check(stream=None, device=None) -> tuple[int, int]:
+    """Synchronise the stream and read/clear the device status word.
+    Returns (status, site)."""
+    lib = load_library()
+    device = device if device is not None else torch.cuda.current_device()
+    site = ctypes.c_int(0)
+    with torch.cuda.device(device):
+        rc = lib.attn_jvp_check(_stream_handle(device, stream), ctypes.byref(site))
+    return rc, site.value

@@ -1,0 +1,123 @@
+/*
+ * attn_jvp.h -- C ABI of the B200 (sm_100a) attention forward + JVP library.
+ *
+ * The operation.  The FlashAttention-2 JVP kernel of rCM ("Large Scale
+ * Diffusion Distillation via Score-Regularized Continuous-Time Consistency",
+ * ai.info AI summary, Key Contributions 1 and Methodology in Plain English;
+ * papernotes.org notes, 关键设计 1) folds the Jacobian-vector product into the
+ * attention forward pass, for self- and cross-attention, and carries the
+ * tangents through the same block-wise tiling.  For every batch b, head h and
+ * query row i, over the valid keys j < n_b:
+ *
+ *     S_ij  = scale * q_i . k_j                 P = softmax_j(S)
+ *     O_i   = sum_j P_ij v_j                    lse_i = ln sum_j exp(S_ij)
+ *     S'_ij = scale * (q'_i . k_j + q_i . k'_j)
+ *     O'_i  = sum_j P_ij (S'_ij - mu_i) v_j + sum_j P_ij v'_j,
+ *             mu_i = sum_j P_ij S'_ij
+ *
+ * i.e. O' = P'V + PV' with P' = P (S' - mu), the exact directional
+ * derivative of O along (Q', K', V').  The scale has no tangent.
+ *
+ * Layout.  Every tensor is dense, contiguous and row-major in device memory:
+ *     q, q_dot, o, o_dot : bf16 [B, H, Lq, d]
+ *     k, k_dot, v, v_dot : bf16 [B, H, Lk, d]
+ *     lse                : fp32 [B, H, Lq]
+ *     kv_len             : int32 [B] or NULL
+ * K and V have the same head count as Q.  bf16 is the IEEE-754 binary32 upper
+ * half; outputs are rounded to nearest even from fp32 accumulators.
+ *
+ * Masking.  n_b = min(Lk, kv_len[b]) clamped below at 0; with kv_len == NULL,
+ * n_b = Lk.  Keys j >= n_b take no part in any output: their k, k', v, v'
+ * may hold any bits (NaN included).  A row with n_b == 0 gets O = O' = 0 and
+ * lse = -inf.  kv_len is read on the device, so its values are not checked
+ * on the host.  There is no causal mask.
+ *
+ * Ownership.  The caller owns every buffer.  The library allocates no device
+ * memory, keeps no per-call state, and returns as soon as the work is queued
+ * on `stream` (asynchronous).  Outputs must not overlap inputs or each other.
+ *
+ * Errors.  Argument errors are detected on the host before anything is
+ * queued; outputs are then left untouched.  Failures that only the device
+ * can see (a pipeline wait that gave up) are recorded in a per-device status
+ * word and reported by attn_jvp_check().
+ */
+#ifndef ATTN_JVP_H
+#define ATTN_JVP_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_JVP_OK = 0,
+    ATTN_JVP_ERR_NULL = -1,    /* a required pointer is NULL                         */
+    ATTN_JVP_ERR_SHAPE = -2,   /* B, H, Lq or Lk < 1, or a size past the limits below  */
+    ATTN_JVP_ERR_HEADDIM = -3, /* d is not 64 or 128                                  */
+    ATTN_JVP_ERR_ALIGN = -4,   /* a tensor pointer is not 16-byte aligned             */
+    ATTN_JVP_ERR_LAUNCH = -5,  /* the CUDA runtime refused the launch or a query      */
+    ATTN_JVP_ERR_TIMEOUT = -6, /* a device-side wait gave up (see attn_jvp_check)    */
+    ATTN_JVP_ERR_VALUE = -7    /* scale not finite, or outputs overlap inputs         */
+} attn_jvp_status;
+
+/*
+ * attn_jvp_fwd -- queue O, O' and lse for the whole [B, H] batch on `stream`.
+ *
+ *   q, k, v              bf16 device pointers (layout above)
+ *   q_dot, k_dot, v_dot  bf16 device pointers, the tangents Q', K', V'
+ *   o, o_dot             bf16 device pointers, written
+ *   lse                  fp32 device pointer, written (natural log)
+ *   B, H, Lq, Lk         >= 1; B*H*Lq and B*H*Lk below 2^31; Lq, Lk below 2^31
+ *   d                    64 or 128
+ *   scale                finite; the usual choice is 1/sqrt(d)
+ *   kv_len               device int32[B] or NULL
+ *   stream               a cudaStream_t, or NULL for the legacy default stream
+ *
+ * Returns ATTN_JVP_OK once the kernel is queued, or a negative status.
+ * Thread-safe; the first call on a device also sets that device's kernel
+ * attributes.
+ */
+int attn_jvp_fwd(const void *q, const void *k, const void *v,
+                 const void *q_dot, const void *k_dot, const void *v_dot,
+                 void *o, void *o_dot, float *lse,
+                 int B, int H, int Lq, int Lk, int d, float scale,
+                 const int32_t *kv_len, void *stream);
+
+/*
+ * attn_jvp_check -- synchronise `stream`, then read and clear the current
+ * device's status word.  Returns ATTN_JVP_OK, ATTN_JVP_ERR_TIMEOUT if a
+ * kernel launched since the last check gave up on a pipeline wait (its
+ * outputs are then unspecified), or ATTN_JVP_ERR_LAUNCH if the
+ * synchronisation itself failed.  If `site` is not NULL it receives the code
+ * of the first wait that gave up (0 if none).
+ */
+int attn_jvp_check(void *stream, int *site);
+
+/* Static English text for a status code. */
+const char *attn_jvp_status_string(int status);
+
+/*
+ * attn_jvp_fwd_debug -- test hook: attn_jvp_fwd with an explicit wait limit
+ * and fault-injection flags, so a test can make a device-side wait run out
+ * without hanging or faulting the GPU.
+ *   timeout_ns  limit for every device-side wait (0 = the default, 2 s)
+ *   flags       ATTN_JVP_DEBUG_* bits; 0 behaves exactly like attn_jvp_fwd
+ * No counterpart on the pages: it exists to test the failure path.
+ */
+#define ATTN_JVP_DEBUG_STARVE_Q 1 /* never load Q/Q': the first wait on it runs out */
+int attn_jvp_fwd_debug(const void *q, const void *k, const void *v,
+                       const void *q_dot, const void *k_dot, const void *v_dot,
+                       void *o, void *o_dot, float *lse,
+                       int B, int H, int Lq, int Lk, int d, float scale,
+                       const int32_t *kv_len, void *stream,
+                       uint64_t timeout_ns, int flags);
+
+/* Library version, for logs: major*10000 + minor*100 + patch. */
+int attn_jvp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_JVP_H */
