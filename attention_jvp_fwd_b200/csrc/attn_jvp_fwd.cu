@@ -12,10 +12,11 @@
 //     K' sit next to each other in shared memory, so Q [K ; K']^T is a single
 //     N = 128 MMA that writes S and Q K'^T side by side; Q' K^T then adds onto
 //     the second half.  Together this is the K = 2d product [Q | Q'][K' | K]^T;
-//   * one warpgroup (thread = query row) runs the online softmax in registers:
-//     running max m (lazily rescaled), denominator l = sum p and
-//     a = sum p (s S'_raw - c).  It writes P and P * (s S'_raw - c) back into
-//     TMEM as bf16 over the S columns;
+//   * two warpgroups run the online softmax in registers, thread = query row,
+//     each on one half of the tile's 64 key columns; they exchange partial row
+//     maxima through shared memory.  Running max m (lazily rescaled),
+//     denominator l = sum p and a = sum p (s S'_raw - c).  They write P and
+//     P * (s S'_raw - c) back into TMEM as bf16 over the S columns;
 //   * O += P V and O'_acc += [P(sS' - c) | P] [V ; V'] are tcgen05 MMAs with A
 //     read from TMEM;
 //   * the epilogue forms O = O_acc / l and O' = (O'_acc - (a / l) O_acc) / l.
@@ -46,9 +47,11 @@ namespace ajvp {
 
 constexpr int BM = 128;                   // query rows per CTA (= TMEM lanes)
 constexpr int BN = 64;                    // keys per K/V tile
-constexpr int NTHREADS = 192;             // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr int NTHREADS = 320;             // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
+constexpr int NSOFT = 256;                // softmax threads: two warpgroups
+constexpr int BAR_SOFT = 1;               // named barrier of the softmax warpgroups
 constexpr uint32_t TMEM_COLS = 512;
-constexpr float RESCALE_THRESHOLD = 8.0f; // log2 units: rescale when the max grows by 2^8
+constexpr float RESCALE_THRESHOLD = 4.0f; // log2 units: rescale when the max grows by 2^4
 constexpr uint64_t DEFAULT_TIMEOUT_NS = 2000000000ull;
 
 // Wait sites recorded in the status word when a wait gives up.
@@ -63,6 +66,7 @@ enum : int {
     SITE_O_DONE = 8,
     SITE_V_TAIL = 9,
     SITE_DRAIN = 10,
+    SITE_SMEM_ALIGN = 11,
 };
 
 template <int D>
@@ -80,11 +84,16 @@ struct Cfg {
     static constexpr uint32_t OFF_BAR = OFF_V + NV * VST_BYTES;
     static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 2 + 1 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + base alignment slack
-    // TMEM columns: O | O'_acc | S buffer 0 (S, S'_raw) | S buffer 1
+    static constexpr uint32_t OFF_XCH = OFF_MISC + 16;            // float [2][2][128]
+    static constexpr uint32_t SMEM_BYTES = OFF_XCH + 2 * 2 * 128 * 4;
+    // TMEM columns: O | O'_acc | S buffer 0 (S, S'_raw) | S buffer 1.  Inside an S
+    // buffer, bf16 P goes to columns [16, 48) and P (sS' - c) to [80, 112):
+    // each softmax warpgroup then overwrites only columns it has read itself.
     static constexpr uint32_t T_O = 0;
     static constexpr uint32_t T_OD = D;
     static constexpr uint32_t T_S = 2 * D;
+    static constexpr uint32_t T_P = 16;       // offset of bf16 P inside an S buffer
+    static constexpr uint32_t T_PD = BN + 16; // offset of bf16 P (sS' - c)
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, 2 * BN, false);
     static constexpr uint32_t IDESC_SD = idesc_bf16_f32(BM, BN, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
@@ -140,9 +149,14 @@ template <int D>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_constant__ Params p)
 {
     using C = Cfg<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    extern __shared__ __align__(1024) uint8_t smem[];
+    // The 128-byte swizzle atoms must start on 1024-byte boundaries.  The
+    // dynamic window is 1024-aligned in practice; if it ever is not, record it
+    // and do nothing rather than compute garbage.
+    if (smem_addr(smem) & 1023u) {
+        if (threadIdx.x == 0) atomicCAS(&g_status, 0, SITE_SMEM_ALIGN);
+        return;
+    }
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -180,7 +194,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
-            mbar_init(&p_full[s], 128);
+            mbar_init(&p_full[s], NSOFT);
         }
         mbar_init(o_done, 1);
         mbar_init(drain, 1);
@@ -274,11 +288,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             if (ok) tc_fence_after();
             const uint32_t qa = smem_addr(smem + C::OFF_Q);
             const uint32_t qda = smem_addr(smem + C::OFF_QD);
-            for (int j = 0; j <= nT && ok; ++j) {
-                if (j < nT) {
+            // S_js and PV_jp are issued in whichever order their inputs arrive,
+            // with S at most one tile ahead of PV (S_js overwrites the buffer
+            // that held P_{js-2}, so PV_{js-2} must already be issued).  A late
+            // K tile then never holds back a PV whose P is ready.
+            int js = 0, jp = 0, polls = 0;
+            uint64_t t_last = globaltimer_ns();
+            while (ok && jp < nT) {
+                bool progressed = false;
+                if (js < nT && js <= jp + 1 &&
+                    mbar_test_wait(smem_addr(&k_full[js % C::NK]), (js / C::NK) & 1)) {
+                    const int j = js;
                     const int s = j % C::NK;
-                    ok = wait_bar(&k_full[s], (j / C::NK) & 1, wc, SITE_K_FULL);
-                    if (!ok) break;
                     tc_fence_after();
                     const uint32_t tS = tbase + C::T_S + (j & 1) * (2 * BN);
                     const uint32_t ka = smem_addr(smem + C::OFF_K + s * C::KST_BYTES);
@@ -301,14 +322,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     mma_commit(&k_empty[s]);
                     mma_commit(&s_full[j & 1]);
                     issued = true;
-                }
-                if (j >= 1) {
-                    const int jj = j - 1;
+                    ++js;
+                    progressed = true;
+                } else if (jp < js && mbar_test_wait(smem_addr(&p_full[jp & 1]), (jp >> 1) & 1) &&
+                           mbar_test_wait(smem_addr(&v_full[jp % C::NV]), (jp / C::NV) & 1)) {
+                    const int jj = jp;
                     const int s = jj % C::NV;
-                    ok = wait_bar(&p_full[jj & 1], (jj >> 1) & 1, wc, SITE_P_FULL);
-                    if (!ok) break;
-                    ok = wait_bar(&v_full[s], (jj / C::NV) & 1, wc, SITE_V_FULL);
-                    if (!ok) break;
                     tc_fence_after();
                     const uint32_t tP = tbase + C::T_S + (jj & 1) * (2 * BN);
                     const uint32_t va = smem_addr(smem + C::OFF_V + s * C::VST_BYTES);
@@ -316,21 +335,37 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     // O += P V
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(tbase + C::T_O, tP + kk * 8, sdesc_sw128(va + kk * 2048, BN * 128, 1024),
-                               C::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts(tbase + C::T_O, tP + C::T_P + kk * 8,
+                               sdesc_sw128(va + kk * 2048, BN * 128, 1024), C::IDESC_PV,
+                               (jj > 0 || kk > 0) ? 1u : 0u);
                     // O'_acc += P(sS' - c) V
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(tbase + C::T_OD, tP + BN + kk * 8,
+                        mma_ts(tbase + C::T_OD, tP + C::T_PD + kk * 8,
                                sdesc_sw128(va + kk * 2048, BN * 128, 1024), C::IDESC_PV,
                                (jj > 0 || kk > 0) ? 1u : 0u);
                     // O'_acc += P V'
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(tbase + C::T_OD, tP + kk * 8, sdesc_sw128(vda + kk * 2048, BN * 128, 1024),
-                               C::IDESC_PV, 1u);
+                        mma_ts(tbase + C::T_OD, tP + C::T_P + kk * 8,
+                               sdesc_sw128(vda + kk * 2048, BN * 128, 1024), C::IDESC_PV, 1u);
                     mma_commit(&v_empty[s]);
                     mma_commit(o_done);
+                    ++jp;
+                    progressed = true;
+                }
+                if (progressed) {
+                    polls = 0;
+                    t_last = globaltimer_ns();
+                } else if (++polls >= 64) {
+                    polls = 0;
+                    if (*abort_flag) {
+                        ok = false;
+                    } else if (globaltimer_ns() - t_last > p.timeout_ns) {
+                        *abort_flag = 1;
+                        atomicCAS(&g_status, 0, js < nT && js <= jp + 1 ? SITE_K_FULL : SITE_P_FULL);
+                        ok = false;
+                    }
                 }
             }
             if (!ok && issued) {
@@ -341,62 +376,78 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
+        // Two warpgroups, thread = query row.  Warpgroup g owns key columns
+        // [32g, 32g + 32) of every tile; at the end it writes output g
+        // (0: O and lse, 1: O').
+        const int g = (warp - 2) >> 2;
         const int quad = warp & 3;  // TMEM lane quadrant this warp may touch
         const int r = quad * 32 + lane;
-        const int st = tid - 64;
+        const int gt = tid - 64 - g * 128;  // thread index inside the warpgroup
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int grow = q0 + r;
         const size_t orow = (static_cast<size_t>(bh) * p.Lq + grow) * D;
-        __nv_bfloat16 *o_ptr = static_cast<__nv_bfloat16 *>(p.o) + orow;
-        __nv_bfloat16 *od_ptr = static_cast<__nv_bfloat16 *>(p.od) + orow;
+        __nv_bfloat16 *out_ptr = static_cast<__nv_bfloat16 *>(g == 0 ? p.o : p.od) + orow;
+        float *xch = reinterpret_cast<float *>(smem + C::OFF_XCH);  // [slot][warpgroup][row]
 
         if (nT == 0) {
             if (grow < p.Lq) {
                 const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-                for (int c = 0; c < D / 8; ++c) {
-                    reinterpret_cast<uint4 *>(o_ptr)[c] = z;
-                    reinterpret_cast<uint4 *>(od_ptr)[c] = z;
-                }
-                p.lse[static_cast<size_t>(bh) * p.Lq + grow] = -INFINITY;
+                for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4 *>(out_ptr)[c] = z;
+                if (g == 0) p.lse[static_cast<size_t>(bh) * p.Lq + grow] = -INFINITY;
             }
         } else {
             const float sl2 = p.sl2;
             const float sc = p.scale;
             const bool neg = sl2 < 0.f;
-            float m_used = -INFINITY, l = 0.f, acc_a = 0.f, cctr = 0.f;
+            const int c0 = 32 * g;
+            // l: sum of the rounded P the MMAs use (normalises O, O');
+            // le: exact fp32 sum of p (for lse); acc_a: sum of rounded P (sS' - c)
+            float m_used = -INFINITY, l = 0.f, le = 0.f, acc_a = 0.f, cctr = 0.f;
             bool ok = true;
             for (int j = 0; j < nT; ++j) {
                 const int bsel = j & 1;
-                ok = __all_sync(0xffffffffu, wait_bar(&s_full[bsel], (j >> 1) & 1, wc, SITE_S_FULL));
-                if (!ok) break;
-                tc_fence_after();
                 const uint32_t tS = tbase + lane_off + C::T_S + bsel * (2 * BN);
-                uint32_t ra[32], rb[32];
-                tmem_ld32(tS, ra);
-                tmem_ld32(tS + 32, rb);
-                tmem_ld_wait2(ra, rb);
-                float x[BN];
+                const bool got = wait_bar(&s_full[bsel], (j >> 1) & 1, wc, SITE_S_FULL);
+                tc_fence_after();
+                uint32_t ra[32];
+                tmem_ld32(tS + c0, ra);
+                tmem_ld_wait(ra);
+                float x[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    x[i] = u2f(ra[i]);
-                    x[32 + i] = u2f(rb[i]);
-                }
-                const int valid = nb - j * BN;  // >= 1
-                const bool tail = valid < BN;
+                for (int i = 0; i < 32; ++i) x[i] = u2f(ra[i]);
+                const int valid = nb - j * BN - c0;  // valid columns of this half
+                const bool tail = valid < 32;
                 if (tail) {
                     const float pad = neg ? INFINITY : -INFINITY;
 #pragma unroll
-                    for (int i = 0; i < BN; ++i) x[i] = (i < valid) ? x[i] : pad;
+                    for (int i = 0; i < 32; ++i) x[i] = (i < valid) ? x[i] : pad;
                 }
-                float mx = x[0];
+                float e0 = x[0], e1 = x[1], e2 = x[2], e3 = x[3];
                 if (neg) {
 #pragma unroll
-                    for (int i = 1; i < BN; ++i) mx = fminf(mx, x[i]);
+                    for (int i = 4; i < 32; i += 4) {
+                        e0 = fminf(e0, x[i]);
+                        e1 = fminf(e1, x[i + 1]);
+                        e2 = fminf(e2, x[i + 2]);
+                        e3 = fminf(e3, x[i + 3]);
+                    }
+                    e0 = fminf(fminf(e0, e1), fminf(e2, e3));
                 } else {
 #pragma unroll
-                    for (int i = 1; i < BN; ++i) mx = fmaxf(mx, x[i]);
+                    for (int i = 4; i < 32; i += 4) {
+                        e0 = fmaxf(e0, x[i]);
+                        e1 = fmaxf(e1, x[i + 1]);
+                        e2 = fmaxf(e2, x[i + 2]);
+                        e3 = fmaxf(e3, x[i + 3]);
+                    }
+                    e0 = fmaxf(fmaxf(e0, e1), fmaxf(e2, e3));
                 }
+                xch[(j & 1) * 256 + g * 128 + r] = e0;
+                ok = bar_and(BAR_SOFT, NSOFT, got);
+                if (!ok) break;
+                const float eo = xch[(j & 1) * 256 + (g ^ 1) * 128 + r];
+                const float mx = neg ? fminf(e0, eo) : fmaxf(e0, eo);
                 const float m_tile = mx * sl2;
                 float alpha = 1.f;
                 bool rescale = false;
@@ -408,122 +459,178 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     rescale = true;
                 }
                 l *= alpha;
+                le *= alpha;
                 acc_a *= alpha;
                 const float nm = -m_used;
-                float ps = 0.f;
 #pragma unroll
-                for (int i = 0; i < BN; ++i) {
-                    x[i] = ex2_approx(fmaf(x[i], sl2, nm));
-                    ps += x[i];
+                for (int i = 0; i < 32; ++i) x[i] = ex2_approx(fmaf(x[i], sl2, nm));
+                if (tail) {
+                    // padded keys: p = 0 exactly (the pad times a zero scale is NaN)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = (i < valid) ? x[i] : 0.f;
                 }
-                l += ps;
-
-                uint32_t da[32], db[32];
-                tmem_ld32(tS + BN, da);
-                tmem_ld32(tS + BN + 32, db);
-                tmem_ld_wait2(da, db);
+                {
+                    float e0 = 0.f, e1 = 0.f, e2 = 0.f, e3 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        e0 += x[i];
+                        e1 += x[i + 1];
+                        e2 += x[i + 2];
+                        e3 += x[i + 3];
+                    }
+                    le += (e0 + e1) + (e2 + e3);
+                }
+                uint32_t rd[32];
+                tmem_ld32(tS + BN + c0, rd);
+                tmem_ld_wait(rd);
                 if (j == 0) {
-                    float num = 0.f;
+                    // centring constant: p-weighted mean of s S' over the first
+                    // keys of the first tile (warpgroup 0's half, which always
+                    // holds a valid key), shared with warpgroup 1
+                    if (g == 0) {
+                        float n0 = 0.f, n1 = 0.f, n2 = 0.f, n3 = 0.f;
 #pragma unroll
-                    for (int i = 0; i < BN; ++i) {
-                        const float sd = u2f(i < 32 ? da[i] : db[i - 32]) * sc;
-                        num += (tail && i >= valid) ? 0.f : x[i] * sd;
+                        for (int i = 0; i < 32; i += 4) {
+                            n0 += (tail && i >= valid) ? 0.f : x[i] * (u2f(rd[i]) * sc);
+                            n1 += (tail && i + 1 >= valid) ? 0.f : x[i + 1] * (u2f(rd[i + 1]) * sc);
+                            n2 += (tail && i + 2 >= valid) ? 0.f : x[i + 2] * (u2f(rd[i + 2]) * sc);
+                            n3 += (tail && i + 3 >= valid) ? 0.f : x[i + 3] * (u2f(rd[i + 3]) * sc);
+                        }
+                        float pw = 0.f;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) pw += x[i];
+                        cctr = ((n0 + n1) + (n2 + n3)) / pw;
+                        xch[128 + r] = cctr;  // slot 0, warpgroup 1's entry: already read
                     }
-                    cctr = num / ps;
+                    bar_sync(BAR_SOFT, NSOFT);
+                    if (g == 1) cctr = xch[128 + r];
                 }
-                uint32_t pk[32], pdk[32];
-                float asum = 0.f;
+                // bf16 operands of the PV MMAs.  l and a sum exactly these rounded
+                // values, so O = sum(P V) / sum(P) is normalised by the weights
+                // the tensor core used; the rounding error then enters O' only
+                // through (v_j - O), which is small for the dominant keys.
+                uint32_t pk[16], pdk[16];
+                float s0 = 0.f, s1 = 0.f, a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int c0 = 2 * i, c1 = 2 * i + 1;
-                    const float s0 = fmaf(u2f(c0 < 32 ? da[c0] : db[c0 - 32]), sc, -cctr);
-                    const float s1 = fmaf(u2f(c1 < 32 ? da[c1] : db[c1 - 32]), sc, -cctr);
-                    float d0 = x[c0] * s0;
-                    float d1 = x[c1] * s1;
+                for (int i = 0; i < 16; ++i) {
+                    const int k0 = 2 * i, k1 = 2 * i + 1;
+                    float d0 = x[k0] * fmaf(u2f(rd[k0]), sc, -cctr);
+                    float d1 = x[k1] * fmaf(u2f(rd[k1]), sc, -cctr);
                     if (tail) {
-                        d0 = (c0 < valid) ? d0 : 0.f;
-                        d1 = (c1 < valid) ? d1 : 0.f;
+                        d0 = (k0 < valid) ? d0 : 0.f;
+                        d1 = (k1 < valid) ? d1 : 0.f;
                     }
-                    asum += d0 + d1;
-                    pk[i] = pack_bf16x2(x[c0], x[c1]);
-                    pdk[i] = pack_bf16x2(d0, d1);
+                    const uint32_t u0 = round_bf16_bits(x[k0]), u1 = round_bf16_bits(x[k1]);
+                    const uint32_t w0 = round_bf16_bits(d0), w1 = round_bf16_bits(d1);
+                    pk[i] = __byte_perm(u0, u1, 0x7632);
+                    pdk[i] = __byte_perm(w0, w1, 0x7632);
+                    const float ps2 = u2f(u0 & 0xFFFF0000u) + u2f(u1 & 0xFFFF0000u);
+                    const float pd2 = u2f(w0 & 0xFFFF0000u) + u2f(w1 & 0xFFFF0000u);
+                    if (i & 1) {
+                        s1 += ps2;
+                        a1 += pd2;
+                    } else {
+                        s0 += ps2;
+                        a0 += pd2;
+                    }
                 }
-                acc_a += asum;
+                l += s0 + s1;
+                acc_a += a0 + a1;
 
                 if (j >= 1) {
-                    // PV of the previous tile must be done before O may be rescaled;
-                    // every phase of o_done is observed in order.
-                    ok = __all_sync(0xffffffffu, wait_bar(o_done, (j - 1) & 1, wc, SITE_O_DONE));
+                    // PV of the previous tile must be done before O may be
+                    // rescaled; every phase of o_done is observed in order.
+                    const bool done = wait_bar(o_done, (j - 1) & 1, wc, SITE_O_DONE);
+                    ok = bar_and(BAR_SOFT, NSOFT, done);
                     if (!ok) break;
                     tc_fence_after();
                 }
                 if (__any_sync(0xffffffffu, rescale)) {
+                    const uint32_t tacc = tbase + lane_off + (g == 0 ? C::T_O : C::T_OD);
 #pragma unroll 1
-                    for (int c = 0; c < 2 * D; c += 32) {
+                    for (int c = 0; c < D; c += 32) {
                         uint32_t t[32];
-                        tmem_ld32(tbase + lane_off + C::T_O + c, t);
+                        tmem_ld32(tacc + c, t);
                         tmem_ld_wait(t);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) t[i] = f2u(u2f(t[i]) * alpha);
-                        tmem_st32(tbase + lane_off + C::T_O + c, t);
+                        tmem_st32(tacc + c, t);
                     }
                 }
-                if (tail) {
-                    // Zero the V and V' rows of padded keys so their bits (NaN
-                    // included) cannot reach the P V products.
+                const int vt = nb - j * BN;  // valid keys in the tile
+                if (vt < BN) {
+                    // Zero the V (g = 0) / V' (g = 1) rows of padded keys so
+                    // their bits (NaN included) cannot reach the PV products.
                     const int s = j % C::NV;
-                    ok = __all_sync(0xffffffffu, wait_bar(&v_full[s], (j / C::NV) & 1, wc, SITE_V_TAIL));
+                    const bool landed = wait_bar(&v_full[s], (j / C::NV) & 1, wc, SITE_V_TAIL);
+                    ok = bar_and(BAR_SOFT, NSOFT, landed);
                     if (!ok) break;
-                    uint8_t *vst = smem + C::OFF_V + s * C::VST_BYTES;
-                    const int nrow = BN - valid;
+                    uint8_t *vst = smem + C::OFF_V + s * C::VST_BYTES + g * (C::NKB * BN * 128);
+                    const int nrow = BN - vt;
                     const int per_blk = nrow * 8;
-                    const int chunks = 2 * C::NKB * per_blk;
-                    for (int idx = st; idx < chunks; idx += 128) {
+                    const int chunks = C::NKB * per_blk;
+                    for (int idx = gt; idx < chunks; idx += 128) {
                         const int blk = idx / per_blk;
                         const int rem = idx - blk * per_blk;
-                        const int row = valid + (rem >> 3);
+                        const int row = vt + (rem >> 3);
                         *reinterpret_cast<uint4 *>(vst + blk * (BN * 128) + row * 128 + (rem & 7) * 16) =
                             make_uint4(0, 0, 0, 0);
                     }
                     fence_proxy_async_smem();
                 }
-                tmem_st32(tS, pk);
-                tmem_st32(tS + BN, pdk);
+                tmem_st16(tS + C::T_P + 16 * g, pk);
+                tmem_st16(tS + C::T_PD + 16 * g, pdk);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&p_full[bsel]);
             }
-            if (ok) ok = __all_sync(0xffffffffu, wait_bar(o_done, (nT - 1) & 1, wc, SITE_O_DONE));
+            if (ok) {
+                const bool done = wait_bar(o_done, (nT - 1) & 1, wc, SITE_O_DONE);
+                ok = bar_and(BAR_SOFT, NSOFT, done);
+            }
             if (ok) {
                 tc_fence_after();
-                const float inv_l = 1.f / l;
-                const float coef = acc_a * inv_l;
+                // The sums are split across the two warpgroups.  Warpgroup 0
+                // needs the totals of l and le, warpgroup 1 those of l and a;
+                // both add the two halves of l in the same order.
+                xch[g * 128 + r] = l;
+                xch[256 + g * 128 + r] = (g == 0) ? acc_a : le;
+                bar_sync(BAR_SOFT, NSOFT);
+                const float lt = xch[r] + xch[128 + r];
+                const float inv_l = 1.f / lt;
+                const float at = (g == 1) ? xch[256 + r] + acc_a : 0.f;
+                const float let = (g == 0) ? le + xch[256 + 128 + r] : 0.f;
+                const float coef = at * inv_l;
+                const uint32_t to = tbase + lane_off + C::T_O;
+                const uint32_t tod = tbase + lane_off + C::T_OD;
 #pragma unroll 1
                 for (int c = 0; c < D; c += 32) {
                     uint32_t ov[32], odv[32];
-                    tmem_ld32(tbase + lane_off + C::T_O + c, ov);
-                    tmem_ld32(tbase + lane_off + C::T_OD + c, odv);
-                    tmem_ld_wait2(ov, odv);
-                    uint32_t po[16], pod[16];
+                    uint32_t pv[16];
+                    if (g == 0) {
+                        tmem_ld32(to + c, ov);
+                        tmem_ld_wait(ov);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float a0 = u2f(ov[2 * i]), a1 = u2f(ov[2 * i + 1]);
-                        const float b0 = u2f(odv[2 * i]), b1 = u2f(odv[2 * i + 1]);
-                        po[i] = pack_bf16x2(a0 * inv_l, a1 * inv_l);
-                        pod[i] = pack_bf16x2(fmaf(-coef, a0, b0) * inv_l, fmaf(-coef, a1, b1) * inv_l);
+                        for (int i = 0; i < 16; ++i)
+                            pv[i] = pack_bf16x2(u2f(ov[2 * i]) * inv_l, u2f(ov[2 * i + 1]) * inv_l);
+                    } else {
+                        tmem_ld32(to + c, ov);
+                        tmem_ld32(tod + c, odv);
+                        tmem_ld_wait2(ov, odv);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pv[i] = pack_bf16x2(fmaf(-coef, u2f(ov[2 * i]), u2f(odv[2 * i])) * inv_l,
+                                                fmaf(-coef, u2f(ov[2 * i + 1]), u2f(odv[2 * i + 1])) * inv_l);
                     }
                     if (grow < p.Lq) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(o_ptr + c);
-                        uint4 *dsd = reinterpret_cast<uint4 *>(od_ptr + c);
+                        uint4 *dst = reinterpret_cast<uint4 *>(out_ptr + c);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            dst[i] = make_uint4(po[4 * i], po[4 * i + 1], po[4 * i + 2], po[4 * i + 3]);
-                            dsd[i] = make_uint4(pod[4 * i], pod[4 * i + 1], pod[4 * i + 2], pod[4 * i + 3]);
-                        }
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pv[4 * i], pv[4 * i + 1], pv[4 * i + 2], pv[4 * i + 3]);
                     }
                 }
-                if (grow < p.Lq)
-                    p.lse[static_cast<size_t>(bh) * p.Lq + grow] = (m_used + log2f(l)) * 0.69314718055994531f;
+                if (g == 0 && grow < p.Lq)
+                    p.lse[static_cast<size_t>(bh) * p.Lq + grow] = (m_used + log2f(let)) * 0.69314718055994531f;
             }
         }
     }

@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention forward + JVP on B200.
+
+One step = one call of the whole path (one kernel launch) over one batch of a
+named synthetic workload (default: T2I self-attention, B=2 H=16 L=4096
+d=128).  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl ours|reference] [--no-cpu-baseline]
+
+Metric: TFLOP/s counted as 12 * Lq * Lk * d per (b, h), over the valid keys.
+Multi-GPU (torchrun): every rank runs its own copy of the workload (seed =
+rank), no collective on the data path ("weak" scaling); value = all ranks'
+FLOPs / the slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded
+row sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("attention fwd+JVP TFLOP/s (12·Lq·Lk·d/head) and % of B200 BF16 "
+          "dense peak")
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
+KERNEL_SOURCES = ["attention_jvp_fwd_b200/csrc/attn_jvp_fwd.cu",
+                  "attention_jvp_fwd_b200/csrc/sm100.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="t2i_self")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--e2e-steps", type=int, default=0, help="0 = min(steps, 100)")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------- helpers
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), float(pk["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_PEAKS["bf16_tflops"], FALLBACK_PEAKS["hbm_gbs"], "fallback"
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on
+    the current kernel source (else None)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = t.get(workload)
+    if not e or e.get("source_sha256") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def algorithmic_bytes(w) -> float:
+    """Bytes the method must move per launch: read Q, Q' and the valid rows of
+    K, K', V, V' once, write O, O' (bf16) and lse (fp32)."""
+    BH = w.B * w.H
+    n_valid = (np.clip(w.kv_len, 0, w.Lk).astype(np.int64) * w.H).sum() if w.kv_len is not None \
+        else BH * w.Lk
+    return float(2 * w.d * (2 * BH * w.Lq + 4 * n_valid) + 4 * BH * w.Lq * w.d + 4 * BH * w.Lq)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{self.gpu_index}.csv")
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    rows.append({"sm": float(parts[2]), "max": float(parts[3]),
+                                 "power": float(parts[4]),
+                                 "hw": parts[6], "hw_th": parts[7], "sw_th": parts[8],
+                                 "sw_pc": parts[9]})
+                except ValueError:
+                    continue
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for k, name in (("hw", "hw_slowdown"), ("hw_th", "hw_thermal_slowdown"),
+                            ("sw_th", "sw_thermal_slowdown"), ("sw_pc", "sw_power_cap")):
+                if r[k].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([r["sm"] for r in load])),
+                "sm_max_mhz": float(max(r["max"] for r in rows)),
+                "reasons": sorted(reasons), "samples": len(load)}
+
+
+# ----------------------------------------------------------------- distributed
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def aggregate(local_ms: float, local_flops: float, group_active: bool, device=None):
+    """Max of the per-rank times and sum of the per-rank FLOPs across ranks."""
+    if not group_active:
+        return local_ms, local_flops
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    f = torch.tensor([local_flops], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(f, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(f.item())
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def time_oracle(w, seconds: float, seed: int = 123):
+    """Time the fp64 oracle on a row sample sized for about `seconds`."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    total_rows = w.B * w.H * w.Lq
+    cores = oracle.max_threads()
+    probe = min(total_rows, max(cores * 2, 16))
+    rows = np.sort(rng.choice(total_rows, size=probe, replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.attn_jvp(*w.inputs(), w.scale, kv_len=w.kv_len, rows=rows)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    n = int(min(total_rows, max(probe, probe * seconds / dt)))
+    rows = np.sort(rng.choice(total_rows, size=n, replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.attn_jvp(*w.inputs(), w.scale, kv_len=w.kv_len, rows=rows)
+    dt = time.perf_counter() - t0
+    flops = row_flops(w, rows)
+    return flops / dt / 1e12, cores, n, dt
+
+
+def row_flops(w, rows) -> float:
+    b = (np.asarray(rows) // (w.H * w.Lq)).astype(np.int64)
+    n = np.full(b.shape, w.Lk, np.int64) if w.kv_len is None else \
+        np.clip(w.kv_len.astype(np.int64)[b], 0, w.Lk)
+    return float(12.0 * w.d * n.sum())
+
+
+def run_reference(args):
+    ws, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    import oracle
+    from attention_jvp_fwd_b200 import workloads as W
+    w = W.make(args.workload, seed=args.seed)
+    total_rows = w.B * w.H * w.Lq
+    cores = oracle.max_threads()
+    rng = np.random.default_rng(7)
+    # calibrate the cost of one row, then size every step so the whole
+    # warm-up + timed run stays near `budget` seconds
+    probe = np.sort(rng.choice(total_rows, size=min(total_rows, 2 * cores), replace=False))
+    t0 = time.perf_counter()
+    oracle.attn_jvp(*w.inputs(), w.scale, kv_len=w.kv_len, rows=probe)
+    per_row = (time.perf_counter() - t0) / len(probe)
+    budget = 120.0
+    rows_per_step = int(max(1, min(total_rows, budget / (args.steps + args.warmup) / per_row)))
+    samples = [np.sort(rng.choice(total_rows, size=rows_per_step, replace=False))
+               for _ in range(args.steps + args.warmup)]
+    for s in samples[:args.warmup]:
+        oracle.attn_jvp(*w.inputs(), w.scale, kv_len=w.kv_len, rows=s)
+    flops = 0.0
+    t0 = time.perf_counter()
+    for s in samples[args.warmup:]:
+        oracle.attn_jvp(*w.inputs(), w.scale, kv_len=w.kv_len, rows=s)
+        flops += row_flops(w, s)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = (f"{rows_per_step} random query rows per step of {args.workload} "
+              f"(of {total_rows}), all keys of each row; fp64 oracle, OpenMP")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, args),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, args):
+    in_bytes = 2 * w.d * (2 * w.B * w.H * w.Lq + 4 * w.B * w.H * w.Lk)
+    return {"workload": w.name, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
+            "scale": w.scale, "kv_len": None if w.kv_len is None else w.kv_len.tolist(),
+            "seed": args.seed, "input_bytes": in_bytes,
+            "l2": ("inputs exceed L2 (%.0f MB > 126 MB), no flush" % (in_bytes / 1e6))
+            if in_bytes > L2_BYTES else "L2 flushed between steps"}
+
+
+# ----------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_setup()
+    group = ws > 1
+    if group:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from attention_jvp_fwd_b200.build import build
+    if rank == 0 or not group:
+        build()
+    if group:
+        dist.barrier()
+    import attention_jvp_fwd_b200 as A
+    from attention_jvp_fwd_b200 import workloads as W
+
+    w = W.make(args.workload, seed=args.seed + rank)
+    host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+            for x in w.inputs()]
+    ins = [h.to(dev, non_blocking=True) for h in host]
+    kv = torch.from_numpy(w.kv_len).to(dev) if w.kv_len is not None else None
+    B, H, Lq, d = w.B, w.H, w.Lq, w.d
+    o = torch.empty((B, H, Lq, d), dtype=torch.bfloat16, device=dev)
+    od = torch.empty_like(o)
+    lse = torch.empty((B, H, Lq), dtype=torch.float32, device=dev)
+    in_bytes = sum(x.numel() * 2 for x in ins)
+    flush = None
+    if in_bytes <= L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    flops_step = w.flops_valid()
+
+    def step():
+        A.attn_jvp_fwd(*ins, scale=w.scale, kv_len=kv, out=(o, od, lse), stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+            if flush is not None:
+                flush.zero_()
+    torch.cuda.synchronize(dev)
+    st, site = A.attn_jvp_check(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} at site {site} after warm-up")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.6)
+    if group:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev = []
+    if flush is None:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        kernel_ms_total = e0.elapsed_time(e1)
+    else:
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                flush.zero_()
+                a.record(stream)
+                step()
+                b.record(stream)
+                ev.append((a, b))
+        torch.cuda.synchronize(dev)
+        kernel_ms_total = sum(a.elapsed_time(b) for a, b in ev)
+    if group:
+        dist.barrier()
+    clocks = sampler.stop()
+    st, site = A.attn_jvp_check(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} at site {site} in the timed region")
+
+    local_ms = kernel_ms_total
+    max_ms, total_flops = aggregate(local_ms, flops_step * args.steps, group, dev)
+    value = total_flops / (max_ms * 1e-3) / 1e12
+
+    # end to end: pinned host inputs -> device, kernel, outputs -> pinned host
+    e2e_steps = args.e2e_steps or min(args.steps, 100)
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hod = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    torch.cuda.synchronize(dev)
+    if group:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(e2e_steps):
+            for dst, src in zip(ins, host):
+                dst.copy_(src, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hod.copy_(od, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms, e2e_flops = aggregate(e0.elapsed_time(e1), flops_step * e2e_steps, group, dev)
+    e2e_value = e2e_flops / (e2e_ms * 1e-3) / 1e12
+    h2d = in_bytes
+    d2h = (o.numel() + od.numel()) * 2 + lse.numel() * 4
+
+    peak_tf, peak_hbm, peak_src = load_peaks()
+    per_launch_ms = local_ms / args.steps
+    achieved = flops_step / (per_launch_ms * 1e-3) / 1e12
+    traffic = measured_traffic(args.workload)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, args),
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf,
+                     "peak_source": f"{peak_src} bf16 dense (burst)", "unit": UNIT,
+                     "frac": achieved / peak_tf, "traffic": traffic,
+                     "algorithmic_bytes": algorithmic_bytes(w),
+                     "flops_per_launch": flops_step,
+                     "kernel": f"attn_jvp_fwd_kernel<{d}>"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "clocks": clocks,
+    }
+    if w.kv_len is not None:
+        line["config"]["flops_nominal_per_step"] = w.flops_nominal()
+    if rank == 0 and not group and not args.no_cpu_baseline:
+        v, cores, n, dt = time_oracle(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"{n} random query rows of {w.name} (all keys), "
+                                          f"{dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if group:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

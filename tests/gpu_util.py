@@ -47,8 +47,9 @@ def ratio(err_max, ref_max):
 
 def compare(g, ref, what=""):
     """Returns a dict of metrics; asserts the parity bar."""
-    go, god, gl = g
-    ro, rod, rl = ref
+    d = g[0].shape[-1]
+    go, god, gl = tuple(np.asarray(x).reshape(-1, d) for x in g[:2]) + (np.asarray(g[2]).reshape(-1),)
+    ro, rod, rl = tuple(np.asarray(x).reshape(-1, d) for x in ref[:2]) + (np.asarray(ref[2]).reshape(-1),)
     eo = ratio(np.max(np.abs(go - ro)), np.max(np.abs(ro)))
     eod = ratio(np.max(np.abs(god - rod)), np.max(np.abs(rod)))
     fin = np.isfinite(rl)

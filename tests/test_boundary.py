@@ -1,0 +1,89 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from attention_jvp_fwd_b200 import api
+from attention_jvp_fwd_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_jvp.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return api.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(attn_jvp_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_abi():
+    assert set(declared_functions()) >= {"attn_jvp_fwd", "attn_jvp_check",
+                                         "attn_jvp_status_string"}
+
+
+def test_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"library does not export {name}"
+    assert set(api.EXPORTED) == set(declared_functions())
+
+
+def _call(lib, ptrs=None, B=1, H=1, Lq=1, Lk=1, d=64, scale=0.125, kv=None):
+    if ptrs is None:
+        ptrs = [0x10000 * (i + 1) for i in range(9)]
+    return lib.attn_jvp_fwd(*[ctypes.c_void_p(p) for p in ptrs], B, H, Lq, Lk, d,
+                            ctypes.c_float(scale), kv, None)
+
+
+def test_argument_errors(lib):
+    good = [0x100000 * (i + 1) for i in range(9)]
+    for i in range(9):
+        bad = list(good)
+        bad[i] = 0
+        assert _call(lib, bad) == api.ATTN_JVP_ERR_NULL
+    for shape in [(0, 1, 1, 1), (1, 0, 1, 1), (1, 1, 0, 1), (1, 1, 1, 0), (1, 1, -5, 1)]:
+        assert _call(lib, good, *shape) == api.ATTN_JVP_ERR_SHAPE
+    assert _call(lib, good, 1 << 16, 1 << 16, 1, 1) == api.ATTN_JVP_ERR_SHAPE
+    for d in (0, 32, 96, 256):
+        assert _call(lib, good, d=d) == api.ATTN_JVP_ERR_HEADDIM
+    for i in range(8):
+        bad = list(good)
+        bad[i] += 8
+        assert _call(lib, bad) == api.ATTN_JVP_ERR_ALIGN
+    bad = list(good)
+    bad[8] += 2
+    assert _call(lib, bad) == api.ATTN_JVP_ERR_ALIGN
+    assert _call(lib, good, kv=ctypes.c_void_p(0x1002)) == api.ATTN_JVP_ERR_ALIGN
+    for s in (float("nan"), float("inf")):
+        assert _call(lib, good, scale=s) == api.ATTN_JVP_ERR_VALUE
+    alias = list(good)
+    alias[6] = alias[0]  # o == q
+    assert _call(lib, alias) == api.ATTN_JVP_ERR_VALUE
+    alias = list(good)
+    alias[7] = alias[6] + 64  # o and o_dot overlap (each holds 1*1*1*64 bf16 = 128 bytes)
+    assert _call(lib, alias) == api.ATTN_JVP_ERR_VALUE
+
+
+def test_status_strings(lib):
+    for code in range(-7, 1):
+        s = api.attn_jvp_status_string(code)
+        assert s and s != "unknown status"
+    assert api.attn_jvp_status_string(42) == "unknown status"
+    assert lib.attn_jvp_version() >= 100
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        api.attn_jvp_fwd(q, q, q, q, q, q)
+    with pytest.raises(TypeError):
+        api.attn_jvp_fwd(q.float(), q, q, q, q, q)
