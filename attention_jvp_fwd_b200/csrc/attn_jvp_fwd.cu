@@ -47,8 +47,7 @@ namespace ajvp {
 
 constexpr int BM = 128;                   // query rows per CTA (= TMEM lanes)
 constexpr int BN = 64;                    // keys per K/V tile
-constexpr int NTHREADS = 320;             // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
-constexpr int NSOFT = 256;                // softmax threads: two warpgroups
+constexpr int NSOFT = 256;                // softmax threads: two warpgroups (warps 2-9)
 constexpr int BAR_SOFT = 1;               // named barrier of the softmax warpgroups
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 4.0f; // log2 units: rescale when the max grows by 2^4
@@ -69,22 +68,43 @@ enum : int {
     SITE_SMEM_ALIGN = 11,
 };
 
-template <int D>
+// Two launch shapes share one kernel body:
+//  - single CTA (PAIR = false): the CTA computes its own 128 x N MMAs;
+//  - CTA pair (PAIR = true, d = 128): a cluster of two CTAs owns two adjacent
+//    128-row query tiles of one (b, h); the leader issues M = 256 MMAs that
+//    read A and write D in both CTAs while each CTA stages only half of every
+//    B operand.  Per tile the leader loads K and the first 32 rows of K, the
+//    peer loads K' and the last 32 rows of K, and each loads its 64-column half
+//    of V and V'.  That halves the B-operand shared-memory reads, the TMA
+//    writes and the L2 reads per SM.
+template <int D, bool PAIR>
 struct Cfg {
+    static_assert(!PAIR || D == 128, "the CTA-pair layout splits V by 64-column halves of d = 128");
     static constexpr int NKB = D / 64;               // 128-byte column blocks per row
-    static constexpr int NK = (D == 128) ? 3 : 4;    // K/K' ring depth
-    static constexpr int NV = (D == 128) ? 2 : 4;    // V/V' ring depth
-    static constexpr uint32_t Q_BYTES = BM * D * 2;  // one of Q, Q'
-    static constexpr uint32_t KST_BYTES = 2 * BN * D * 2;
-    static constexpr uint32_t VST_BYTES = 2 * BN * D * 2;
+    static constexpr int NTHREADS = PAIR ? 352 : 320;  // + relay warp 10 in pair mode
+    static constexpr int NCTA = PAIR ? 2 : 1;
+    static constexpr int NK = PAIR ? 4 : ((D == 128) ? 3 : 4);  // K ring depth
+    static constexpr int NV = PAIR ? 4 : ((D == 128) ? 2 : 4);  // V ring depth
+    static constexpr uint32_t Q_BYTES = BM * D * 2;  // one of Q, Q' (per CTA)
+    // K stage.  Single CTA: K then K' rows in each column block (one 128-row
+    // operand [K; K']).  Pair: X (K in the leader, K' in the peer; 64 rows)
+    // then Z (32 rows of K).
+    static constexpr uint32_t X_BYTES = BN * D * 2;
+    static constexpr uint32_t Z_BYTES = (BN / 2) * D * 2;
+    static constexpr uint32_t KST_BYTES = PAIR ? X_BYTES + Z_BYTES : 2 * BN * D * 2;
+    // V stage: V then V' (pair: this CTA's 64-column half of each)
+    static constexpr uint32_t VHALF_BYTES = PAIR ? BN * 64 * 2 : BN * D * 2;
+    static constexpr uint32_t VST_BYTES = 2 * VHALF_BYTES;
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_QD = Q_BYTES;
     static constexpr uint32_t OFF_K = 2 * Q_BYTES;
     static constexpr uint32_t OFF_V = OFF_K + NK * KST_BYTES;
     static constexpr uint32_t OFF_BAR = OFF_V + NV * VST_BYTES;
-    static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 2 + 1 + 1;
+    // q_full, k_full[NK], k_empty[NK], v_full[NV], v_ready[NV], v_empty[NV],
+    // s_full[2], p_full[2], o_done, drain
+    static constexpr int NBAR = 1 + 2 * NK + 3 * NV + 2 + 2 + 1 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr uint32_t OFF_XCH = OFF_MISC + 16;            // float [2][2][128]
+    static constexpr uint32_t OFF_XCH = OFF_MISC + 16;  // float [2][2][128]
     static constexpr uint32_t SMEM_BYTES = OFF_XCH + 2 * 2 * 128 * 4;
     // TMEM columns: O | O'_acc | S buffer 0 (S, S'_raw) | S buffer 1.  Inside an S
     // buffer, bf16 P goes to columns [16, 48) and P (sS' - c) to [80, 112):
@@ -92,17 +112,19 @@ struct Cfg {
     static constexpr uint32_t T_O = 0;
     static constexpr uint32_t T_OD = D;
     static constexpr uint32_t T_S = 2 * D;
-    static constexpr uint32_t T_P = 16;       // offset of bf16 P inside an S buffer
-    static constexpr uint32_t T_PD = BN + 16; // offset of bf16 P (sS' - c)
-    static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, 2 * BN, false);
-    static constexpr uint32_t IDESC_SD = idesc_bf16_f32(BM, BN, false);
-    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
+    static constexpr uint32_t T_P = 16;        // offset of bf16 P inside an S buffer
+    static constexpr uint32_t T_PD = BN + 16;  // offset of bf16 P (sS' - c)
+    static constexpr int MMA_M = BM * NCTA;
+    static constexpr uint32_t IDESC_S = idesc_bf16_f32(MMA_M, 2 * BN, false);
+    static constexpr uint32_t IDESC_SD = idesc_bf16_f32(MMA_M, BN, false);
+    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(MMA_M, D, true);
+    static constexpr int P_ARRIVALS = 8 * NCTA;  // one per softmax warp
     static_assert(T_S + 4 * BN <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct Params {
-    CUtensorMap tm_q, tm_qd, tm_k, tm_kd, tm_v, tm_vd;
+    CUtensorMap tm_q, tm_qd, tm_k, tm_kd, tm_v, tm_vd, tm_k32;
     void *o;
     void *od;
     float *lse;
@@ -123,16 +145,18 @@ struct WaitCtx {
 
 // Bounded wait for phase `parity` of `bar`.  Returns false if the limit ran
 // out (recording `site`) or, when honor_abort is set, if another role gave up.
+// cluster_scope: acquire at cluster scope (barriers the peer CTA signals).
 __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, const WaitCtx &c, int site,
-                                      bool honor_abort = true)
+                                      bool honor_abort = true, bool cluster_scope = false)
 {
     const uint32_t a = smem_addr(bar);
-    if (mbar_try_wait(a, parity)) return true;
+    auto probe = [&]() { return cluster_scope ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity); };
+    if (probe()) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(a, parity)) return true;
+            if (probe()) return true;
         if (honor_abort && *c.abort) return false;
         if (globaltimer_ns() - t0 > c.limit_ns) {
             *c.abort = 1;
@@ -142,17 +166,28 @@ __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, const Wait
     }
 }
 
+// One inline probe before falling back to the bounded loop.
+__device__ __forceinline__ bool wait_bar_fast(uint64_t *bar, uint32_t parity, const WaitCtx &c, int site,
+                                              bool cluster_scope)
+{
+    const uint32_t a = smem_addr(bar);
+    if (cluster_scope ? mbar_test_wait_cluster(a, parity) : mbar_test_wait(a, parity)) return true;
+    return wait_bar(bar, parity, c, site, true, cluster_scope);
+}
+
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 __device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
 
-template <int D>
-__global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_constant__ Params p)
+template <int D, bool PAIR>
+__global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
+    attn_jvp_fwd_kernel(const __grid_constant__ Params p)
 {
-    using C = Cfg<D>;
+    using C = Cfg<D, PAIR>;
     extern __shared__ __align__(1024) uint8_t smem[];
     // The 128-byte swizzle atoms must start on 1024-byte boundaries.  The
     // dynamic window is 1024-aligned in practice; if it ever is not, record it
-    // and do nothing rather than compute garbage.
+    // and do nothing rather than compute garbage (both CTAs of a pair see the
+    // same layout, so both return here).
     if (smem_addr(smem) & 1023u) {
         if (threadIdx.x == 0) atomicCAS(&g_status, 0, SITE_SMEM_ALIGN);
         return;
@@ -161,8 +196,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int qt = blockIdx.x % p.nqt;
-    const int bh = blockIdx.x / p.nqt;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    int qt, bh;
+    if constexpr (PAIR) {
+        const int nqp = (p.nqt + 1) >> 1;  // query-tile pairs per (b, h)
+        const int pair = blockIdx.x >> 1;
+        qt = 2 * (pair % nqp) + static_cast<int>(rank);
+        bh = pair / nqp;
+    } else {
+        qt = blockIdx.x % p.nqt;
+        bh = blockIdx.x / p.nqt;
+    }
     const int b = bh / p.H;
     const int q0 = qt * BM;
     int nb = p.Lk;
@@ -174,7 +219,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
     uint64_t *k_full = q_full + 1;
     uint64_t *k_empty = k_full + C::NK;
     uint64_t *v_full = k_empty + C::NK;
-    uint64_t *v_empty = v_full + C::NV;
+    uint64_t *v_ready = v_full + C::NV;
+    uint64_t *v_empty = v_ready + C::NV;
     uint64_t *s_full = v_empty + C::NV;
     uint64_t *p_full = s_full + 2;
     uint64_t *o_done = p_full + 2;
@@ -190,11 +236,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         }
         for (int s = 0; s < C::NV; ++s) {
             mbar_init(&v_full[s], 1);
+            mbar_init(&v_ready[s], C::NCTA);
             mbar_init(&v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
-            mbar_init(&p_full[s], NSOFT);
+            mbar_init(&p_full[s], C::P_ARRIVALS);
         }
         mbar_init(o_done, 1);
         mbar_init(drain, 1);
@@ -208,16 +255,33 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         tma_prefetch_desc(&p.tm_kd);
         tma_prefetch_desc(&p.tm_v);
         tma_prefetch_desc(&p.tm_vd);
+        if (PAIR) tma_prefetch_desc(&p.tm_k32);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(tmem_slot, TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (PAIR) {
+        cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+    } else {
+        __syncthreads();
+    }
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const WaitCtx wc{abort_flag, p.timeout_ns};
+    // cluster addresses of the leader's barriers that both CTAs signal
+    const uint32_t q_full_lead = PAIR ? mapa_shared(smem_addr(q_full), 0) : smem_addr(q_full);
+    const uint32_t k_full_lead = PAIR ? mapa_shared(smem_addr(k_full), 0) : smem_addr(k_full);
+    const uint32_t v_ready_lead = PAIR ? mapa_shared(smem_addr(v_ready), 0) : smem_addr(v_ready);
+    const uint32_t p_full_lead = PAIR ? mapa_shared(smem_addr(p_full), 0) : smem_addr(p_full);
+    (void)v_ready_lead;
+    (void)p_full_lead;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -226,12 +290,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const uint64_t pol_kv = l2_policy_evict_last();
             const bool load_q = !(p.flags & ATTN_JVP_DEBUG_STARVE_Q);
             if (load_q) {
-                mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
+                if constexpr (PAIR) {
+                    // the leader's barrier counts both CTAs' Q and Q' bytes
+                    if (leader) mbar_arrive_expect_tx(q_full, 2 * 2 * C::Q_BYTES);
 #pragma unroll
-                for (int c = 0; c < C::NKB; ++c) {
-                    tma_load_3d(smem + C::OFF_Q + c * BM * 128, &p.tm_q, q_full, c * 64, q0, bh, pol_q);
-                    tma_load_3d(smem + C::OFF_QD + c * BM * 128, &p.tm_qd, q_full, c * 64, q0, bh,
-                                pol_q);
+                    for (int c = 0; c < C::NKB; ++c) {
+                        tma_load_3d_pair(smem + C::OFF_Q + c * BM * 128, &p.tm_q, q_full_lead, c * 64, q0, bh,
+                                         pol_q);
+                        tma_load_3d_pair(smem + C::OFF_QD + c * BM * 128, &p.tm_qd, q_full_lead, c * 64, q0,
+                                         bh, pol_q);
+                    }
+                } else {
+                    mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NKB; ++c) {
+                        tma_load_3d(smem + C::OFF_Q + c * BM * 128, &p.tm_q, q_full, c * 64, q0, bh, pol_q);
+                        tma_load_3d(smem + C::OFF_QD + c * BM * 128, &p.tm_qd, q_full, c * 64, q0, bh,
+                                    pol_q);
+                    }
                 }
             }
             int nk = 0, nv = 0;
@@ -239,40 +315,66 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             for (int j = 0; j <= nT && ok; ++j) {
                 if (j < nT) {
                     const int s = j % C::NK;
-                    if (j >= C::NK) ok = wait_bar(&k_empty[s], ((j / C::NK) - 1) & 1, wc, SITE_K_EMPTY);
+                    if (j >= C::NK)
+                        ok = wait_bar(&k_empty[s], ((j / C::NK) - 1) & 1, wc, SITE_K_EMPTY, true, PAIR);
                     if (!ok) break;
                     uint8_t *dst = smem + C::OFF_K + s * C::KST_BYTES;
-                    mbar_arrive_expect_tx(&k_full[s], C::KST_BYTES);
+                    if constexpr (PAIR) {
+                        if (leader) mbar_arrive_expect_tx(&k_full[s], 2 * C::KST_BYTES);
+                        const uint32_t bar = k_full_lead + s * 8;
+                        const CUtensorMap *mx = leader ? &p.tm_k : &p.tm_kd;
 #pragma unroll
-                    for (int c = 0; c < C::NKB; ++c) {
-                        tma_load_3d(dst + c * (2 * BN * 128), &p.tm_k, &k_full[s], c * 64, j * BN, bh,
-                                    pol_kv);
-                        tma_load_3d(dst + c * (2 * BN * 128) + BN * 128, &p.tm_kd, &k_full[s], c * 64,
-                                    j * BN, bh, pol_kv);
+                        for (int c = 0; c < C::NKB; ++c) {
+                            tma_load_3d_pair(dst + c * (BN * 128), mx, bar, c * 64, j * BN, bh, pol_kv);
+                            tma_load_3d_pair(dst + C::X_BYTES + c * (BN / 2 * 128), &p.tm_k32, bar, c * 64,
+                                             j * BN + static_cast<int>(rank) * (BN / 2), bh, pol_kv);
+                        }
+                    } else {
+                        mbar_arrive_expect_tx(&k_full[s], C::KST_BYTES);
+#pragma unroll
+                        for (int c = 0; c < C::NKB; ++c) {
+                            tma_load_3d(dst + c * (2 * BN * 128), &p.tm_k, &k_full[s], c * 64, j * BN, bh,
+                                        pol_kv);
+                            tma_load_3d(dst + c * (2 * BN * 128) + BN * 128, &p.tm_kd, &k_full[s], c * 64,
+                                        j * BN, bh, pol_kv);
+                        }
                     }
                     ++nk;
                 }
                 if (j >= 1) {
                     const int jj = j - 1;
                     const int s = jj % C::NV;
-                    if (jj >= C::NV) ok = wait_bar(&v_empty[s], ((jj / C::NV) - 1) & 1, wc, SITE_V_EMPTY);
+                    if (jj >= C::NV)
+                        ok = wait_bar(&v_empty[s], ((jj / C::NV) - 1) & 1, wc, SITE_V_EMPTY, true, PAIR);
                     if (!ok) break;
                     uint8_t *dst = smem + C::OFF_V + s * C::VST_BYTES;
                     mbar_arrive_expect_tx(&v_full[s], C::VST_BYTES);
+                    if constexpr (PAIR) {
+                        // this CTA's 64-column half of V and V' (local barrier)
+                        const int c0 = static_cast<int>(rank) * 64;
+                        tma_load_3d(dst, &p.tm_v, &v_full[s], c0, jj * BN, bh, pol_kv);
+                        tma_load_3d(dst + C::VHALF_BYTES, &p.tm_vd, &v_full[s], c0, jj * BN, bh, pol_kv);
+                    } else {
 #pragma unroll
-                    for (int c = 0; c < C::NKB; ++c) {
-                        tma_load_3d(dst + c * (BN * 128), &p.tm_v, &v_full[s], c * 64, jj * BN, bh, pol_kv);
-                        tma_load_3d(dst + (C::NKB + c) * (BN * 128), &p.tm_vd, &v_full[s], c * 64, jj * BN,
-                                    bh, pol_kv);
+                        for (int c = 0; c < C::NKB; ++c) {
+                            tma_load_3d(dst + c * (BN * 128), &p.tm_v, &v_full[s], c * 64, jj * BN, bh, pol_kv);
+                            tma_load_3d(dst + (C::NKB + c) * (BN * 128), &p.tm_vd, &v_full[s], c * 64, jj * BN,
+                                        bh, pol_kv);
+                        }
                     }
                     ++nv;
                 }
             }
-            // Let every load this thread issued land before the CTA can exit.
-            if (load_q) wait_bar(q_full, 0, wc, SITE_DRAIN, false);
-            for (int s = 0; s < C::NK && s < nk; ++s) {
-                const int t = s + ((nk - 1 - s) / C::NK) * C::NK;
-                wait_bar(&k_full[s], (t / C::NK) & 1, wc, SITE_DRAIN, false);
+            // Let every load land before the CTA can exit.  In a pair the K
+            // and Q bytes of both CTAs are counted on the leader's barriers,
+            // so the leader waits for them; the final cluster barrier keeps
+            // the peer alive until then.
+            if (load_q && leader) wait_bar(q_full, 0, wc, SITE_DRAIN, false, PAIR);
+            if (leader) {
+                for (int s = 0; s < C::NK && s < nk; ++s) {
+                    const int t = s + ((nk - 1 - s) / C::NK) * C::NK;
+                    wait_bar(&k_full[s], (t / C::NK) & 1, wc, SITE_DRAIN, false, PAIR);
+                }
             }
             for (int s = 0; s < C::NV && s < nv; ++s) {
                 const int t = s + ((nv - 1 - s) / C::NV) * C::NV;
@@ -281,9 +383,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && nT > 0) {
-            bool ok = wait_bar(q_full, 0, wc, SITE_Q_FULL);
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (lane == 0 && nT > 0 && leader) {
+            bool ok = wait_bar(q_full, 0, wc, SITE_Q_FULL, true, PAIR);
             bool issued = false;
             if (ok) tc_fence_after();
             const uint32_t qa = smem_addr(smem + C::OFF_Q);
@@ -294,63 +396,101 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             // K tile then never holds back a PV whose P is ready.
             int js = 0, jp = 0, polls = 0;
             uint64_t t_last = globaltimer_ns();
+            auto test = [&](uint64_t *bar, uint32_t parity) {
+                return PAIR ? mbar_test_wait_cluster(smem_addr(bar), parity)
+                            : mbar_test_wait(smem_addr(bar), parity);
+            };
             while (ok && jp < nT) {
                 bool progressed = false;
-                if (js < nT && js <= jp + 1 &&
-                    mbar_test_wait(smem_addr(&k_full[js % C::NK]), (js / C::NK) & 1)) {
+                if (js < nT && js <= jp + 1 && test(&k_full[js % C::NK], (js / C::NK) & 1)) {
                     const int j = js;
                     const int s = j % C::NK;
                     tc_fence_after();
                     const uint32_t tS = tbase + C::T_S + (j & 1) * (2 * BN);
                     const uint32_t ka = smem_addr(smem + C::OFF_K + s * C::KST_BYTES);
-                    // S | Q K'^T  =  Q [K ; K']^T   (N = 2 BN)
+                    if constexpr (PAIR) {
+                        // S | Q K'^T = Q [K ; K']^T: B rows 0-63 (K) in the leader, 64-127 (K') in the peer
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                        const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
-                        mma_ss(tS, sdesc_sw128(qa + oa, 16, 1024), sdesc_sw128(ka + ob, 16, 1024),
-                               C::IDESC_S, kk > 0 ? 1u : 0u);
-                    }
-                    // += Q' K^T into the second half
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                            const uint32_t ob = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+                            mma_ss_pair(tS, sdesc_sw128(qa + oa, 16, 1024), sdesc_sw128(ka + ob, 16, 1024),
+                                        C::IDESC_S, kk > 0 ? 1u : 0u);
+                        }
+                        // += Q' K^T: B rows 0-31 of K in the leader, 32-63 in the peer
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                        const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
-                        mma_ss(tS + BN, sdesc_sw128(qda + oa, 16, 1024), sdesc_sw128(ka + ob, 16, 1024),
-                               C::IDESC_SD, 1u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                            const uint32_t ob = C::X_BYTES + (kk >> 2) * (BN / 2 * 128) + (kk & 3) * 32;
+                            mma_ss_pair(tS + BN, sdesc_sw128(qda + oa, 16, 1024), sdesc_sw128(ka + ob, 16, 1024),
+                                        C::IDESC_SD, 1u);
+                        }
+                        mma_commit_pair_mc(&k_empty[s], 0x3);
+                        mma_commit_pair_mc(&s_full[j & 1], 0x3);
+                    } else {
+                        // S | Q K'^T  =  Q [K ; K']^T   (N = 2 BN)
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                            const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
+                            mma_ss(tS, sdesc_sw128(qa + oa, 16, 1024), sdesc_sw128(ka + ob, 16, 1024),
+                                   C::IDESC_S, kk > 0 ? 1u : 0u);
+                        }
+                        // += Q' K^T into the second half
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                            const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
+                            mma_ss(tS + BN, sdesc_sw128(qda + oa, 16, 1024), sdesc_sw128(ka + ob, 16, 1024),
+                                   C::IDESC_SD, 1u);
+                        }
+                        mma_commit(&k_empty[s]);
+                        mma_commit(&s_full[j & 1]);
                     }
-                    mma_commit(&k_empty[s]);
-                    mma_commit(&s_full[j & 1]);
                     issued = true;
                     ++js;
                     progressed = true;
-                } else if (jp < js && mbar_test_wait(smem_addr(&p_full[jp & 1]), (jp >> 1) & 1) &&
-                           mbar_test_wait(smem_addr(&v_full[jp % C::NV]), (jp / C::NV) & 1)) {
+                } else if (jp < js && test(&p_full[jp & 1], (jp >> 1) & 1) &&
+                           test(PAIR ? &v_ready[jp % C::NV] : &v_full[jp % C::NV], (jp / C::NV) & 1)) {
                     const int jj = jp;
                     const int s = jj % C::NV;
                     tc_fence_after();
                     const uint32_t tP = tbase + C::T_S + (jj & 1) * (2 * BN);
                     const uint32_t va = smem_addr(smem + C::OFF_V + s * C::VST_BYTES);
-                    const uint32_t vda = va + C::NKB * BN * 128;
-                    // O += P V
+                    const uint32_t vda = va + C::VHALF_BYTES;
+                    // LBO: distance between 64-column blocks of V (single CTA, d = 128);
+                    // a pair CTA holds one block, so it is unused there
+                    constexpr uint32_t LBO = BN * 128;
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(tbase + C::T_O, tP + C::T_P + kk * 8,
-                               sdesc_sw128(va + kk * 2048, BN * 128, 1024), C::IDESC_PV,
-                               (jj > 0 || kk > 0) ? 1u : 0u);
-                    // O'_acc += P(sS' - c) V
+                    for (int kk = 0; kk < BN / 16; ++kk) {  // O += P V
+                        const uint32_t a = tP + C::T_P + kk * 8;
+                        const uint64_t bd = sdesc_sw128(va + kk * 2048, LBO, 1024);
+                        const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+                        if constexpr (PAIR) mma_ts_pair(tbase + C::T_O, a, bd, C::IDESC_PV, acc);
+                        else mma_ts(tbase + C::T_O, a, bd, C::IDESC_PV, acc);
+                    }
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(tbase + C::T_OD, tP + C::T_PD + kk * 8,
-                               sdesc_sw128(va + kk * 2048, BN * 128, 1024), C::IDESC_PV,
-                               (jj > 0 || kk > 0) ? 1u : 0u);
-                    // O'_acc += P V'
+                    for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P(sS' - c) V
+                        const uint32_t a = tP + C::T_PD + kk * 8;
+                        const uint64_t bd = sdesc_sw128(va + kk * 2048, LBO, 1024);
+                        const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+                        if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, bd, C::IDESC_PV, acc);
+                        else mma_ts(tbase + C::T_OD, a, bd, C::IDESC_PV, acc);
+                    }
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(tbase + C::T_OD, tP + C::T_P + kk * 8,
-                               sdesc_sw128(vda + kk * 2048, BN * 128, 1024), C::IDESC_PV, 1u);
-                    mma_commit(&v_empty[s]);
-                    mma_commit(o_done);
+                    for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P V'
+                        const uint32_t a = tP + C::T_P + kk * 8;
+                        const uint64_t bd = sdesc_sw128(vda + kk * 2048, LBO, 1024);
+                        if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, bd, C::IDESC_PV, 1u);
+                        else mma_ts(tbase + C::T_OD, a, bd, C::IDESC_PV, 1u);
+                    }
+                    if constexpr (PAIR) {
+                        mma_commit_pair_mc(&v_empty[s], 0x3);
+                        mma_commit_pair_mc(o_done, 0x3);
+                    } else {
+                        mma_commit(&v_empty[s]);
+                        mma_commit(o_done);
+                    }
                     ++jp;
                     progressed = true;
                 }
@@ -369,12 +509,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 }
             }
             if (!ok && issued) {
-                mma_commit(drain);
-                wait_bar(drain, 0, wc, SITE_DRAIN, false);
+                if constexpr (PAIR) mma_commit_pair_mc(drain, 0x1);
+                else mma_commit(drain);
+                wait_bar(drain, 0, wc, SITE_DRAIN, false, PAIR);
             }
         }
         __syncwarp();
-    } else {
+    } else if (PAIR && warp == 10) {
+        // ------------------------------------------------------------ V relay (pair)
+        // Each CTA's V/V' half lands on a local barrier.  This warp zeroes the
+        // rows of padded keys in the tail tile (their bits, NaN included, must
+        // not reach the PV products) and then tells the leader's MMA warp.
+        bool ok = true;
+        for (int j = 0; j < nT && ok; ++j) {
+            const int s = j % C::NV;
+            const bool landed = wait_bar(&v_full[s], (j / C::NV) & 1, wc, SITE_V_TAIL);
+            ok = __all_sync(0xffffffffu, landed);
+            if (!ok) break;
+            const int vt = nb - j * BN;
+            if (vt < BN) {
+                uint8_t *vst = smem + C::OFF_V + s * C::VST_BYTES;
+                const int chunks = 2 * (BN - vt) * 8;  // 16-byte chunks: V and V' rows vt..BN-1
+                for (int idx = lane; idx < chunks; idx += 32) {
+                    const int half = idx / ((BN - vt) * 8);
+                    const int rem = idx - half * ((BN - vt) * 8);
+                    *reinterpret_cast<uint4 *>(vst + half * C::VHALF_BYTES + (vt + (rem >> 3)) * 128 +
+                                               (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(v_ready_lead + s * 8);
+        }
+    } else if (warp >= 2 && warp < 10) {
         // ------------------------------------------------------------ softmax + epilogue
         // Two warpgroups, thread = query row.  Warpgroup g owns key columns
         // [32g, 32g + 32) of every tile; at the end it writes output g
@@ -401,18 +568,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const float sc = p.scale;
             const bool neg = sl2 < 0.f;
             const int c0 = 32 * g;
-            // l: sum of the rounded P the MMAs use (normalises O, O');
-            // le: exact fp32 sum of p (for lse); acc_a: sum of rounded P (sS' - c)
-            float m_used = -INFINITY, l = 0.f, le = 0.f, acc_a = 0.f, cctr = 0.f;
+            // l: exact fp32 sum of p (normalises O and O', gives lse);
+            // acc_a: sum of the bf16-rounded P (sS' - c) that the MMAs consume,
+            // so the rounding of those operands reaches O' only through
+            // (v_j - O), which is small for the keys that dominate.
+            float m_used = -INFINITY, l = 0.f, acc_a = 0.f, cctr = 0.f;
             bool ok = true;
             for (int j = 0; j < nT; ++j) {
                 const int bsel = j & 1;
                 const uint32_t tS = tbase + lane_off + C::T_S + bsel * (2 * BN);
-                const bool got = wait_bar(&s_full[bsel], (j >> 1) & 1, wc, SITE_S_FULL);
+                const bool got = wait_bar_fast(&s_full[bsel], (j >> 1) & 1, wc, SITE_S_FULL, PAIR);
                 tc_fence_after();
-                uint32_t ra[32];
-                tmem_ld32(tS + c0, ra);
-                tmem_ld_wait(ra);
+                uint32_t ra[32], rd[32];
+                tmem_ld32(tS + c0, ra);       // S columns of this half
+                tmem_ld32(tS + BN + c0, rd);  // S'_raw columns of this half
+                tmem_ld_wait2(ra, rd);
                 float x[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] = u2f(ra[i]);
@@ -423,25 +593,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
 #pragma unroll
                     for (int i = 0; i < 32; ++i) x[i] = (i < valid) ? x[i] : pad;
                 }
-                float e0 = x[0], e1 = x[1], e2 = x[2], e3 = x[3];
+                float e0, e1, e2, e3;
                 if (neg) {
-#pragma unroll
-                    for (int i = 4; i < 32; i += 4) {
-                        e0 = fminf(e0, x[i]);
-                        e1 = fminf(e1, x[i + 1]);
-                        e2 = fminf(e2, x[i + 2]);
-                        e3 = fminf(e3, x[i + 3]);
-                    }
-                    e0 = fminf(fminf(e0, e1), fminf(e2, e3));
+                    e0 = min3f(min3f(x[0], x[1], x[2]), min3f(x[3], x[4], x[5]), fminf(x[6], x[7]));
+                    e1 = min3f(min3f(x[8], x[9], x[10]), min3f(x[11], x[12], x[13]), fminf(x[14], x[15]));
+                    e2 = min3f(min3f(x[16], x[17], x[18]), min3f(x[19], x[20], x[21]), fminf(x[22], x[23]));
+                    e3 = min3f(min3f(x[24], x[25], x[26]), min3f(x[27], x[28], x[29]), fminf(x[30], x[31]));
+                    e0 = min3f(e0, e1, fminf(e2, e3));
                 } else {
-#pragma unroll
-                    for (int i = 4; i < 32; i += 4) {
-                        e0 = fmaxf(e0, x[i]);
-                        e1 = fmaxf(e1, x[i + 1]);
-                        e2 = fmaxf(e2, x[i + 2]);
-                        e3 = fmaxf(e3, x[i + 3]);
-                    }
-                    e0 = fmaxf(fmaxf(e0, e1), fmaxf(e2, e3));
+                    e0 = max3f(max3f(x[0], x[1], x[2]), max3f(x[3], x[4], x[5]), fmaxf(x[6], x[7]));
+                    e1 = max3f(max3f(x[8], x[9], x[10]), max3f(x[11], x[12], x[13]), fmaxf(x[14], x[15]));
+                    e2 = max3f(max3f(x[16], x[17], x[18]), max3f(x[19], x[20], x[21]), fmaxf(x[22], x[23]));
+                    e3 = max3f(max3f(x[24], x[25], x[26]), max3f(x[27], x[28], x[29]), fmaxf(x[30], x[31]));
+                    e0 = max3f(e0, e1, fmaxf(e2, e3));
                 }
                 xch[(j & 1) * 256 + g * 128 + r] = e0;
                 ok = bar_and(BAR_SOFT, NSOFT, got);
@@ -459,88 +623,88 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     rescale = true;
                 }
                 l *= alpha;
-                le *= alpha;
                 acc_a *= alpha;
-                const float nm = -m_used;
+                // p = 2^(s * log2(e) * S - m), in pairs
+                {
+                    const uint64_t sl22 = f2_pack(sl2, sl2);
+                    const uint64_t nm2 = f2_pack(-m_used, -m_used);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = ex2_approx(fmaf(x[i], sl2, nm));
+                    for (int i = 0; i < 16; ++i) {
+                        float t0, t1;
+                        f2_unpack(f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), sl22, nm2), t0, t1);
+                        x[2 * i] = ex2_approx(t0);
+                        x[2 * i + 1] = ex2_approx(t1);
+                    }
+                }
                 if (tail) {
                     // padded keys: p = 0 exactly (the pad times a zero scale is NaN)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) x[i] = (i < valid) ? x[i] : 0.f;
                 }
                 {
-                    float e0 = 0.f, e1 = 0.f, e2 = 0.f, e3 = 0.f;
+                    uint64_t s0 = f2_pack(x[0], x[1]), s1 = f2_pack(x[2], x[3]);
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        e0 += x[i];
-                        e1 += x[i + 1];
-                        e2 += x[i + 2];
-                        e3 += x[i + 3];
+                    for (int i = 2; i < 16; i += 2) {
+                        s0 = f2_add(s0, f2_pack(x[2 * i], x[2 * i + 1]));
+                        s1 = f2_add(s1, f2_pack(x[2 * i + 2], x[2 * i + 3]));
                     }
-                    le += (e0 + e1) + (e2 + e3);
+                    float u0, u1, u2, u3;
+                    f2_unpack(s0, u0, u1);
+                    f2_unpack(s1, u2, u3);
+                    l += (u0 + u1) + (u2 + u3);
                 }
-                uint32_t rd[32];
-                tmem_ld32(tS + BN + c0, rd);
-                tmem_ld_wait(rd);
                 if (j == 0) {
                     // centring constant: p-weighted mean of s S' over the first
                     // keys of the first tile (warpgroup 0's half, which always
                     // holds a valid key), shared with warpgroup 1
                     if (g == 0) {
-                        float n0 = 0.f, n1 = 0.f, n2 = 0.f, n3 = 0.f;
+                        float n0 = 0.f, n1 = 0.f, w0 = 0.f, w1 = 0.f;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4) {
+                        for (int i = 0; i < 32; i += 2) {
                             n0 += (tail && i >= valid) ? 0.f : x[i] * (u2f(rd[i]) * sc);
                             n1 += (tail && i + 1 >= valid) ? 0.f : x[i + 1] * (u2f(rd[i + 1]) * sc);
-                            n2 += (tail && i + 2 >= valid) ? 0.f : x[i + 2] * (u2f(rd[i + 2]) * sc);
-                            n3 += (tail && i + 3 >= valid) ? 0.f : x[i + 3] * (u2f(rd[i + 3]) * sc);
+                            w0 += x[i];
+                            w1 += x[i + 1];
                         }
-                        float pw = 0.f;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) pw += x[i];
-                        cctr = ((n0 + n1) + (n2 + n3)) / pw;
+                        cctr = (n0 + n1) / (w0 + w1);
                         xch[128 + r] = cctr;  // slot 0, warpgroup 1's entry: already read
                     }
                     bar_sync(BAR_SOFT, NSOFT);
                     if (g == 1) cctr = xch[128 + r];
                 }
-                // bf16 operands of the PV MMAs.  l and a sum exactly these rounded
-                // values, so O = sum(P V) / sum(P) is normalised by the weights
-                // the tensor core used; the rounding error then enters O' only
-                // through (v_j - O), which is small for the dominant keys.
+                // bf16 operands of the PV MMAs: P and P (s S' - c)
                 uint32_t pk[16], pdk[16];
-                float s0 = 0.f, s1 = 0.f, a0 = 0.f, a1 = 0.f;
+                {
+                    const uint64_t sc2 = f2_pack(sc, sc);
+                    const uint64_t nc2 = f2_pack(-cctr, -cctr);
+                    uint64_t a0 = 0, a1 = 0;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int k0 = 2 * i, k1 = 2 * i + 1;
-                    float d0 = x[k0] * fmaf(u2f(rd[k0]), sc, -cctr);
-                    float d1 = x[k1] * fmaf(u2f(rd[k1]), sc, -cctr);
-                    if (tail) {
-                        d0 = (k0 < valid) ? d0 : 0.f;
-                        d1 = (k1 < valid) ? d1 : 0.f;
+                    for (int i = 0; i < 16; ++i) {
+                        const uint64_t p2 = f2_pack(x[2 * i], x[2 * i + 1]);
+                        const uint64_t d2 = f2_mul(f2_fma(f2_pack(u2f(rd[2 * i]), u2f(rd[2 * i + 1])), sc2, nc2), p2);
+                        float d0, d1;
+                        f2_unpack(d2, d0, d1);
+                        if (tail) {
+                            d0 = (2 * i < valid) ? d0 : 0.f;
+                            d1 = (2 * i + 1 < valid) ? d1 : 0.f;
+                        }
+                        pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+                        pdk[i] = pack_bf16x2(d0, d1);
+                        // the two rounded values as fp32
+                        const uint64_t r2 = f2_pack(u2f(pdk[i] << 16), u2f(pdk[i] & 0xFFFF0000u));
+                        if (i & 1) a1 = f2_add(a1, r2);
+                        else a0 = f2_add(a0, r2);
                     }
-                    const uint32_t u0 = round_bf16_bits(x[k0]), u1 = round_bf16_bits(x[k1]);
-                    const uint32_t w0 = round_bf16_bits(d0), w1 = round_bf16_bits(d1);
-                    pk[i] = __byte_perm(u0, u1, 0x7632);
-                    pdk[i] = __byte_perm(w0, w1, 0x7632);
-                    const float ps2 = u2f(u0 & 0xFFFF0000u) + u2f(u1 & 0xFFFF0000u);
-                    const float pd2 = u2f(w0 & 0xFFFF0000u) + u2f(w1 & 0xFFFF0000u);
-                    if (i & 1) {
-                        s1 += ps2;
-                        a1 += pd2;
-                    } else {
-                        s0 += ps2;
-                        a0 += pd2;
-                    }
+                    float u0, u1, u2, u3;
+                    f2_unpack(a0, u0, u1);
+                    f2_unpack(a1, u2, u3);
+                    acc_a += (u0 + u1) + (u2 + u3);
                 }
-                l += s0 + s1;
-                acc_a += a0 + a1;
 
                 if (j >= 1) {
                     // PV of the previous tile must be done before O may be
                     // rescaled; every phase of o_done is observed in order.
-                    const bool done = wait_bar(o_done, (j - 1) & 1, wc, SITE_O_DONE);
+                    const bool done = wait_bar_fast(o_done, (j - 1) & 1, wc, SITE_O_DONE, PAIR);
                     ok = bar_and(BAR_SOFT, NSOFT, done);
                     if (!ok) break;
                     tc_fence_after();
@@ -558,7 +722,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                 }
                 const int vt = nb - j * BN;  // valid keys in the tile
-                if (vt < BN) {
+                if (!PAIR && vt < BN) {
                     // Zero the V (g = 0) / V' (g = 1) rows of padded keys so
                     // their bits (NaN included) cannot reach the PV products.
                     const int s = j % C::NV;
@@ -582,25 +746,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 tmem_st16(tS + C::T_PD + 16 * g, pdk);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&p_full[bsel]);
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (PAIR) mbar_arrive_cluster(p_full_lead + bsel * 8);
+                    else mbar_arrive(&p_full[bsel]);
+                }
             }
             if (ok) {
-                const bool done = wait_bar(o_done, (nT - 1) & 1, wc, SITE_O_DONE);
+                const bool done = wait_bar(o_done, (nT - 1) & 1, wc, SITE_O_DONE, true, PAIR);
                 ok = bar_and(BAR_SOFT, NSOFT, done);
             }
             if (ok) {
                 tc_fence_after();
-                // The sums are split across the two warpgroups.  Warpgroup 0
-                // needs the totals of l and le, warpgroup 1 those of l and a;
-                // both add the two halves of l in the same order.
+                // l and a are split across the two warpgroups; add the halves
+                // in a fixed order so both see the same totals.
                 xch[g * 128 + r] = l;
-                xch[256 + g * 128 + r] = (g == 0) ? acc_a : le;
+                xch[256 + g * 128 + r] = acc_a;
                 bar_sync(BAR_SOFT, NSOFT);
                 const float lt = xch[r] + xch[128 + r];
                 const float inv_l = 1.f / lt;
-                const float at = (g == 1) ? xch[256 + r] + acc_a : 0.f;
-                const float let = (g == 0) ? le + xch[256 + 128 + r] : 0.f;
-                const float coef = at * inv_l;
+                const float coef = (xch[256 + r] + xch[384 + r]) * inv_l;
                 const uint32_t to = tbase + lane_off + C::T_O;
                 const uint32_t tod = tbase + lane_off + C::T_OD;
 #pragma unroll 1
@@ -630,16 +795,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                 }
                 if (g == 0 && grow < p.Lq)
-                    p.lse[static_cast<size_t>(bh) * p.Lq + grow] = (m_used + log2f(let)) * 0.69314718055994531f;
+                    p.lse[static_cast<size_t>(bh) * p.Lq + grow] = (m_used + log2f(lt)) * 0.69314718055994531f;
             }
         }
     }
 
     tc_fence_before();
-    __syncthreads();
+    if constexpr (PAIR) {
+        // Neither CTA may leave while the leader's MMAs can still read the
+        // peer's shared memory or TMEM, or loads can still signal the leader.
+        cluster_sync();
+    } else {
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tbase, TMEM_COLS);
+        if constexpr (PAIR) tmem_dealloc_pair(tbase, TMEM_COLS);
+        else tmem_dealloc(tbase, TMEM_COLS);
     }
 }
 
@@ -684,7 +856,7 @@ static bool make_map(CUtensorMap *m, const void *base, int D, int L, long long B
 
 constexpr int MAX_DEVICES = 64;
 
-template <int D>
+template <int D, bool PAIR>
 static int prepare_device(int dev)
 {
     static std::mutex mu;
@@ -692,11 +864,36 @@ static int prepare_device(int dev)
     if (dev < 0 || dev >= MAX_DEVICES) return ATTN_JVP_ERR_LAUNCH;
     std::lock_guard<std::mutex> g(mu);
     if (!done[dev]) {
-        if (cudaFuncSetAttribute(attn_jvp_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(Cfg<D>::SMEM_BYTES)) != cudaSuccess)
+        if (cudaFuncSetAttribute(attn_jvp_fwd_kernel<D, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(Cfg<D, PAIR>::SMEM_BYTES)) != cudaSuccess)
             return ATTN_JVP_ERR_LAUNCH;
         done[dev] = true;
     }
+    return ATTN_JVP_OK;
+}
+
+template <int D, bool PAIR>
+static int launch_kernel(const Params &prm, long long grid, cudaStream_t s)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
+    if (int rc = prepare_device<D, PAIR>(dev)) return rc;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(Cfg<D, PAIR>::NTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg<D, PAIR>::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    if (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    if (cudaLaunchKernelEx(&cfg, attn_jvp_fwd_kernel<D, PAIR>, prm) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     return ATTN_JVP_OK;
 }
 
@@ -735,14 +932,19 @@ static int launch(const void *q, const void *k, const void *v, const void *qd, c
     }
 
     const int nqt = (Lq + BM - 1) / BM;
-    const long long grid = static_cast<long long>(nqt) * BH;
+    // One CTA per query tile by default.  The CTA-pair layout (d = 128 only,
+    // selected by a test flag) halves the per-SM operand traffic but couples
+    // the two CTAs' pipelines; on B200 it measures slightly slower today.
+    const bool pair = d == 128 && (flags & ATTN_JVP_DEBUG_CTA_PAIR);
+    const long long grid = pair ? 2ll * ((nqt + 1) / 2) * BH : static_cast<long long>(nqt) * BH;
     if (grid > INT_MAX) return ATTN_JVP_ERR_SHAPE;
 
     Params prm;
     std::memset(&prm, 0, sizeof prm);
     if (!make_map(&prm.tm_q, q, d, Lq, BH, BM) || !make_map(&prm.tm_qd, qd, d, Lq, BH, BM) ||
         !make_map(&prm.tm_k, k, d, Lk, BH, BN) || !make_map(&prm.tm_kd, kd, d, Lk, BH, BN) ||
-        !make_map(&prm.tm_v, v, d, Lk, BH, BN) || !make_map(&prm.tm_vd, vd, d, Lk, BH, BN))
+        !make_map(&prm.tm_v, v, d, Lk, BH, BN) || !make_map(&prm.tm_vd, vd, d, Lk, BH, BN) ||
+        !make_map(&prm.tm_k32, k, d, Lk, BH, BN / 2))
         return ATTN_JVP_ERR_LAUNCH;
     prm.o = o;
     prm.od = od;
@@ -757,16 +959,12 @@ static int launch(const void *q, const void *k, const void *v, const void *qd, c
     prm.timeout_ns = timeout_ns ? timeout_ns : DEFAULT_TIMEOUT_NS;
     prm.flags = flags;
 
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (d == 64) {
-        if (int rc = prepare_device<64>(dev)) return rc;
-        attn_jvp_fwd_kernel<64><<<static_cast<unsigned>(grid), NTHREADS, Cfg<64>::SMEM_BYTES, s>>>(prm);
-    } else {
-        if (int rc = prepare_device<128>(dev)) return rc;
-        attn_jvp_fwd_kernel<128><<<static_cast<unsigned>(grid), NTHREADS, Cfg<128>::SMEM_BYTES, s>>>(prm);
-    }
+    int rc;
+    if (d == 64) rc = launch_kernel<64, false>(prm, grid, s);
+    else if (pair) rc = launch_kernel<128, true>(prm, grid, s);
+    else rc = launch_kernel<128, false>(prm, grid, s);
+    if (rc) return rc;
     if (cudaGetLastError() != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     return ATTN_JVP_OK;
 }
