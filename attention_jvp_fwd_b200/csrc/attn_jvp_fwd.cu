@@ -178,6 +178,34 @@ __device__ __forceinline__ bool wait_bar_fast(uint64_t *bar, uint32_t parity, co
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 __device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
 
+// Max (or min) of the 64 floats held as bits in a and b, as a balanced tree
+// of 3-input operations (32 of them).  Exact, so the order of the two halves
+// does not change the result.
+template <bool MIN>
+__device__ __forceinline__ float row_ext64(const uint32_t (&a)[32], const uint32_t (&b)[32])
+{
+    auto op = [](float x, float y, float z) { return MIN ? min3f(x, y, z) : max3f(x, y, z); };
+    float t[16], u[8], w[4];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) t[i] = op(u2f(a[2 * i]), u2f(a[2 * i + 1]), u2f(b[2 * i]));
+#pragma unroll
+    for (int k = 0; k < 8; ++k) u[k] = op(t[2 * k], t[2 * k + 1], u2f(b[4 * k + 1]));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[k] = op(u[2 * k], u[2 * k + 1], u2f(b[8 * k + 3]));
+    const float y0 = op(w[0], w[1], u2f(b[7]));
+    const float y1 = op(w[2], w[3], u2f(b[23]));
+    const float z = op(y0, y1, u2f(b[15]));
+    return MIN ? fminf(z, u2f(b[31])) : fmaxf(z, u2f(b[31]));
+}
+__device__ __forceinline__ float row_max64(const uint32_t (&a)[32], const uint32_t (&b)[32])
+{
+    return row_ext64<false>(a, b);
+}
+__device__ __forceinline__ float row_min64(const uint32_t (&a)[32], const uint32_t (&b)[32])
+{
+    return row_ext64<true>(a, b);
+}
+
 template <int D, bool PAIR>
 __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
     attn_jvp_fwd_kernel(const __grid_constant__ Params p)
@@ -384,21 +412,30 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader)
-        if (lane == 0 && nT > 0 && leader) {
-            bool ok = wait_bar(q_full, 0, wc, SITE_Q_FULL, true, PAIR);
+        // The whole warp runs this loop (barrier tests and branches are
+        // warp-uniform); one elected lane issues each MMA and commit.
+        if (nT > 0 && leader) {
+            bool ok = __all_sync(0xffffffffu, wait_bar(q_full, 0, wc, SITE_Q_FULL, true, PAIR));
             bool issued = false;
             if (ok) tc_fence_after();
-            const uint32_t qa = smem_addr(smem + C::OFF_Q);
-            const uint32_t qda = smem_addr(smem + C::OFF_QD);
+            // Operand descriptors are built once per buffer; the per-MMA
+            // offsets are added to the start-address field (all shared
+            // addresses fit its 18 bits), which keeps the issue loop short.
+            const uint64_t dq = sdesc_sw128(smem_addr(smem + C::OFF_Q), 16, 1024);
+            const uint64_t dqd = sdesc_sw128(smem_addr(smem + C::OFF_QD), 16, 1024);
             // S_js and PV_jp are issued in whichever order their inputs arrive,
             // with S at most one tile ahead of PV (S_js overwrites the buffer
             // that held P_{js-2}, so PV_{js-2} must already be issued).  A late
             // K tile then never holds back a PV whose P is ready.
+            // The wait limit runs from the first idle check after the last
+            // issue: reading %globaltimer costs hundreds of clocks, so the
+            // issue path never reads it.
             int js = 0, jp = 0, polls = 0;
-            uint64_t t_last = globaltimer_ns();
+            bool idle_timed = false;
+            uint64_t t_idle = 0;
             auto test = [&](uint64_t *bar, uint32_t parity) {
-                return PAIR ? mbar_test_wait_cluster(smem_addr(bar), parity)
-                            : mbar_test_wait(smem_addr(bar), parity);
+                return __all_sync(0xffffffffu, PAIR ? mbar_test_wait_cluster(smem_addr(bar), parity)
+                                                    : mbar_test_wait(smem_addr(bar), parity));
             };
             while (ok && jp < nT) {
                 bool progressed = false;
@@ -407,14 +444,14 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                     const int s = j % C::NK;
                     tc_fence_after();
                     const uint32_t tS = tbase + C::T_S + (j & 1) * (2 * BN);
-                    const uint32_t ka = smem_addr(smem + C::OFF_K + s * C::KST_BYTES);
+                    const uint64_t dk = sdesc_sw128(smem_addr(smem + C::OFF_K + s * C::KST_BYTES), 16, 1024);
                     if constexpr (PAIR) {
                         // S | Q K'^T = Q [K ; K']^T: B rows 0-63 (K) in the leader, 64-127 (K') in the peer
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
                             const uint32_t ob = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-                            mma_ss_pair(tS, sdesc_sw128(qa + oa, 16, 1024), sdesc_sw128(ka + ob, 16, 1024),
+                            mma_ss_pair(tS, desc_add(dq, oa), desc_add(dk, ob),
                                         C::IDESC_S, kk > 0 ? 1u : 0u);
                         }
                         // += Q' K^T: B rows 0-31 of K in the leader, 32-63 in the peer
@@ -422,7 +459,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
                             const uint32_t ob = C::X_BYTES + (kk >> 2) * (BN / 2 * 128) + (kk & 3) * 32;
-                            mma_ss_pair(tS + BN, sdesc_sw128(qda + oa, 16, 1024), sdesc_sw128(ka + ob, 16, 1024),
+                            mma_ss_pair(tS + BN, desc_add(dqd, oa), desc_add(dk, ob),
                                         C::IDESC_SD, 1u);
                         }
                         mma_commit_pair_mc(&k_empty[s], 0x3);
@@ -433,7 +470,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
                             const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
-                            mma_ss(tS, sdesc_sw128(qa + oa, 16, 1024), sdesc_sw128(ka + ob, 16, 1024),
+                            mma_ss(tS, desc_add(dq, oa), desc_add(dk, ob),
                                    C::IDESC_S, kk > 0 ? 1u : 0u);
                         }
                         // += Q' K^T into the second half
@@ -441,7 +478,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
                             const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
-                            mma_ss(tS + BN, sdesc_sw128(qda + oa, 16, 1024), sdesc_sw128(ka + ob, 16, 1024),
+                            mma_ss(tS + BN, desc_add(dqd, oa), desc_add(dk, ob),
                                    C::IDESC_SD, 1u);
                         }
                         mma_commit(&k_empty[s]);
@@ -456,15 +493,15 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                     const int s = jj % C::NV;
                     tc_fence_after();
                     const uint32_t tP = tbase + C::T_S + (jj & 1) * (2 * BN);
-                    const uint32_t va = smem_addr(smem + C::OFF_V + s * C::VST_BYTES);
-                    const uint32_t vda = va + C::VHALF_BYTES;
                     // LBO: distance between 64-column blocks of V (single CTA, d = 128);
                     // a pair CTA holds one block, so it is unused there
                     constexpr uint32_t LBO = BN * 128;
+                    const uint64_t dv = sdesc_sw128(smem_addr(smem + C::OFF_V + s * C::VST_BYTES), LBO, 1024);
+                    const uint64_t dvd = desc_add(dv, C::VHALF_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk) {  // O += P V
                         const uint32_t a = tP + C::T_P + kk * 8;
-                        const uint64_t bd = sdesc_sw128(va + kk * 2048, LBO, 1024);
+                        const uint64_t bd = desc_add(dv, kk * 2048);
                         const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
                         if constexpr (PAIR) mma_ts_pair(tbase + C::T_O, a, bd, C::IDESC_PV, acc);
                         else mma_ts(tbase + C::T_O, a, bd, C::IDESC_PV, acc);
@@ -472,7 +509,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P(sS' - c) V
                         const uint32_t a = tP + C::T_PD + kk * 8;
-                        const uint64_t bd = sdesc_sw128(va + kk * 2048, LBO, 1024);
+                        const uint64_t bd = desc_add(dv, kk * 2048);
                         const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
                         if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, bd, C::IDESC_PV, acc);
                         else mma_ts(tbase + C::T_OD, a, bd, C::IDESC_PV, acc);
@@ -480,7 +517,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P V'
                         const uint32_t a = tP + C::T_P + kk * 8;
-                        const uint64_t bd = sdesc_sw128(vda + kk * 2048, LBO, 1024);
+                        const uint64_t bd = desc_add(dvd, kk * 2048);
                         if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, bd, C::IDESC_PV, 1u);
                         else mma_ts(tbase + C::T_OD, a, bd, C::IDESC_PV, 1u);
                     }
@@ -496,12 +533,16 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                 }
                 if (progressed) {
                     polls = 0;
-                    t_last = globaltimer_ns();
+                    idle_timed = false;
                 } else if (++polls >= 64) {
                     polls = 0;
-                    if (*abort_flag) {
+                    const uint64_t now = __shfl_sync(0xffffffffu, globaltimer_ns(), 0);
+                    if (__any_sync(0xffffffffu, *abort_flag != 0)) {
                         ok = false;
-                    } else if (globaltimer_ns() - t_last > p.timeout_ns) {
+                    } else if (!idle_timed) {
+                        idle_timed = true;
+                        t_idle = now;
+                    } else if (now - t_idle > p.timeout_ns) {
                         *abort_flag = 1;
                         atomicCAS(&g_status, 0, js < nT && js <= jp + 1 ? SITE_K_FULL : SITE_P_FULL);
                         ok = false;
@@ -573,45 +614,44 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
             // so the rounding of those operands reaches O' only through
             // (v_j - O), which is small for the keys that dominate.
             float m_used = -INFINITY, l = 0.f, acc_a = 0.f, cctr = 0.f;
-            bool ok = true;
+            // No named barrier inside the loop: every thread reads the whole
+            // 64-column row of S and forms the same row max, so the two
+            // warpgroups need not meet, and each warp runs through the tiles
+            // at its own pace, coupled only by the MMA barriers.  A wait that
+            // gives up sets `err` and leaves the loop; the barrier after the
+            // loop is reached by all 256 threads either way.
+            bool err = false;
             for (int j = 0; j < nT; ++j) {
                 const int bsel = j & 1;
                 const uint32_t tS = tbase + lane_off + C::T_S + bsel * (2 * BN);
-                const bool got = wait_bar_fast(&s_full[bsel], (j >> 1) & 1, wc, SITE_S_FULL, PAIR);
+                if (!__all_sync(0xffffffffu, wait_bar_fast(&s_full[bsel], (j >> 1) & 1, wc, SITE_S_FULL, PAIR))) {
+                    err = true;
+                    break;
+                }
                 tc_fence_after();
-                uint32_t ra[32], rd[32];
-                tmem_ld32(tS + c0, ra);       // S columns of this half
-                tmem_ld32(tS + BN + c0, rd);  // S'_raw columns of this half
-                tmem_ld_wait2(ra, rd);
-                float x[32];
+                const int vt = nb - j * BN;          // valid keys in the tile
+                const int valid = vt - c0;           // valid columns of this half
+                const bool tail = vt < BN;
+                float mx;
+                uint32_t ra[32];
+                {
+                    uint32_t rb[32];
+                    tmem_ld32(tS + c0, ra);         // S, this half
+                    tmem_ld32(tS + (c0 ^ 32), rb);  // S, the other half (row max only)
+                    tmem_ld_wait2(ra, rb);
+                    if (tail) {
+                        const float pad = neg ? INFINITY : -INFINITY;
+                        const int valid_o = vt - (c0 ^ 32);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = u2f(ra[i]);
-                const int valid = nb - j * BN - c0;  // valid columns of this half
-                const bool tail = valid < 32;
-                if (tail) {
-                    const float pad = neg ? INFINITY : -INFINITY;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] = (i < valid) ? x[i] : pad;
+                        for (int i = 0; i < 32; ++i) {
+                            ra[i] = (i < valid) ? ra[i] : f2u(pad);
+                            rb[i] = (i < valid_o) ? rb[i] : f2u(pad);
+                        }
+                    }
+                    mx = neg ? row_min64(ra, rb) : row_max64(ra, rb);
                 }
-                float e0, e1, e2, e3;
-                if (neg) {
-                    e0 = min3f(min3f(x[0], x[1], x[2]), min3f(x[3], x[4], x[5]), fminf(x[6], x[7]));
-                    e1 = min3f(min3f(x[8], x[9], x[10]), min3f(x[11], x[12], x[13]), fminf(x[14], x[15]));
-                    e2 = min3f(min3f(x[16], x[17], x[18]), min3f(x[19], x[20], x[21]), fminf(x[22], x[23]));
-                    e3 = min3f(min3f(x[24], x[25], x[26]), min3f(x[27], x[28], x[29]), fminf(x[30], x[31]));
-                    e0 = min3f(e0, e1, fminf(e2, e3));
-                } else {
-                    e0 = max3f(max3f(x[0], x[1], x[2]), max3f(x[3], x[4], x[5]), fmaxf(x[6], x[7]));
-                    e1 = max3f(max3f(x[8], x[9], x[10]), max3f(x[11], x[12], x[13]), fmaxf(x[14], x[15]));
-                    e2 = max3f(max3f(x[16], x[17], x[18]), max3f(x[19], x[20], x[21]), fmaxf(x[22], x[23]));
-                    e3 = max3f(max3f(x[24], x[25], x[26]), max3f(x[27], x[28], x[29]), fmaxf(x[30], x[31]));
-                    e0 = max3f(e0, e1, fmaxf(e2, e3));
-                }
-                xch[(j & 1) * 256 + g * 128 + r] = e0;
-                ok = bar_and(BAR_SOFT, NSOFT, got);
-                if (!ok) break;
-                const float eo = xch[(j & 1) * 256 + (g ^ 1) * 128 + r];
-                const float mx = neg ? fminf(e0, eo) : fmaxf(e0, eo);
+                uint32_t rd[32];
+                tmem_ld32(tS + BN + c0, rd);  // S'_raw, this half (waited for below)
                 const float m_tile = mx * sl2;
                 float alpha = 1.f;
                 bool rescale = false;
@@ -624,6 +664,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                 }
                 l *= alpha;
                 acc_a *= alpha;
+                float x[32];
                 // p = 2^(s * log2(e) * S - m), in pairs
                 {
                     const uint64_t sl22 = f2_pack(sl2, sl2);
@@ -631,7 +672,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         float t0, t1;
-                        f2_unpack(f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), sl22, nm2), t0, t1);
+                        f2_unpack(f2_fma(f2_pack(u2f(ra[2 * i]), u2f(ra[2 * i + 1])), sl22, nm2), t0, t1);
                         x[2 * i] = ex2_approx(t0);
                         x[2 * i + 1] = ex2_approx(t1);
                     }
@@ -653,24 +694,45 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                     f2_unpack(s1, u2, u3);
                     l += (u0 + u1) + (u2 + u3);
                 }
+                tmem_ld_wait(rd);
                 if (j == 0) {
-                    // centring constant: p-weighted mean of s S' over the first
-                    // keys of the first tile (warpgroup 0's half, which always
-                    // holds a valid key), shared with warpgroup 1
+                    // centring constant c: the p-weighted mean of s S' over the
+                    // first 32 keys (warpgroup 0's half, which always holds a
+                    // valid key).  Warpgroup 1 forms the same p from the same S
+                    // bits with the same instructions, so both get the same c.
+                    float pc[32], dc[32];
                     if (g == 0) {
-                        float n0 = 0.f, n1 = 0.f, w0 = 0.f, w1 = 0.f;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            n0 += (tail && i >= valid) ? 0.f : x[i] * (u2f(rd[i]) * sc);
-                            n1 += (tail && i + 1 >= valid) ? 0.f : x[i + 1] * (u2f(rd[i + 1]) * sc);
-                            w0 += x[i];
-                            w1 += x[i + 1];
+                        for (int i = 0; i < 32; ++i) {
+                            pc[i] = x[i];
+                            dc[i] = u2f(rd[i]);
                         }
-                        cctr = (n0 + n1) / (w0 + w1);
-                        xch[128 + r] = cctr;  // slot 0, warpgroup 1's entry: already read
+                    } else {
+                        uint32_t cs[32], cdr[32];
+                        tmem_ld32(tS, cs);
+                        tmem_ld32(tS + BN, cdr);
+                        tmem_ld_wait2(cs, cdr);
+                        const uint64_t sl22 = f2_pack(sl2, sl2);
+                        const uint64_t nm2 = f2_pack(-m_used, -m_used);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float t0, t1;
+                            f2_unpack(f2_fma(f2_pack(u2f(cs[2 * i]), u2f(cs[2 * i + 1])), sl22, nm2), t0, t1);
+                            pc[2 * i] = (2 * i < vt) ? ex2_approx(t0) : 0.f;
+                            pc[2 * i + 1] = (2 * i + 1 < vt) ? ex2_approx(t1) : 0.f;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) dc[i] = u2f(cdr[i]);
                     }
-                    bar_sync(BAR_SOFT, NSOFT);
-                    if (g == 1) cctr = xch[128 + r];
+                    float n0 = 0.f, n1 = 0.f, w0 = 0.f, w1 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        n0 = (i >= vt) ? n0 : __fmaf_rn(pc[i], __fmul_rn(dc[i], sc), n0);
+                        n1 = (i + 1 >= vt) ? n1 : __fmaf_rn(pc[i + 1], __fmul_rn(dc[i + 1], sc), n1);
+                        w0 = __fadd_rn(w0, pc[i]);
+                        w1 = __fadd_rn(w1, pc[i + 1]);
+                    }
+                    cctr = __fdiv_rn(__fadd_rn(n0, n1), __fadd_rn(w0, w1));
                 }
                 // bf16 operands of the PV MMAs: P and P (s S' - c)
                 uint32_t pk[16], pdk[16];
@@ -700,13 +762,14 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                     f2_unpack(a1, u2, u3);
                     acc_a += (u0 + u1) + (u2 + u3);
                 }
-
                 if (j >= 1) {
                     // PV of the previous tile must be done before O may be
-                    // rescaled; every phase of o_done is observed in order.
-                    const bool done = wait_bar_fast(o_done, (j - 1) & 1, wc, SITE_O_DONE, PAIR);
-                    ok = bar_and(BAR_SOFT, NSOFT, done);
-                    if (!ok) break;
+                    // rescaled; every warp observes every phase of o_done in
+                    // order (o_done(j) needs this warp's P of tile j).
+                    if (!__all_sync(0xffffffffu, wait_bar_fast(o_done, (j - 1) & 1, wc, SITE_O_DONE, PAIR))) {
+                        err = true;
+                        break;
+                    }
                     tc_fence_after();
                 }
                 if (__any_sync(0xffffffffu, rescale)) {
@@ -721,14 +784,15 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                         tmem_st32(tacc + c, t);
                     }
                 }
-                const int vt = nb - j * BN;  // valid keys in the tile
-                if (!PAIR && vt < BN) {
+                if (!PAIR && tail) {
                     // Zero the V (g = 0) / V' (g = 1) rows of padded keys so
                     // their bits (NaN included) cannot reach the PV products.
+                    // Each warp zeroes its share and fences before it signals P.
                     const int s = j % C::NV;
-                    const bool landed = wait_bar(&v_full[s], (j / C::NV) & 1, wc, SITE_V_TAIL);
-                    ok = bar_and(BAR_SOFT, NSOFT, landed);
-                    if (!ok) break;
+                    if (!__all_sync(0xffffffffu, wait_bar(&v_full[s], (j / C::NV) & 1, wc, SITE_V_TAIL))) {
+                        err = true;
+                        break;
+                    }
                     uint8_t *vst = smem + C::OFF_V + s * C::VST_BYTES + g * (C::NKB * BN * 128);
                     const int nrow = BN - vt;
                     const int per_blk = nrow * 8;
@@ -752,9 +816,11 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                     else mbar_arrive(&p_full[bsel]);
                 }
             }
-            if (ok) {
-                const bool done = wait_bar(o_done, (nT - 1) & 1, wc, SITE_O_DONE, true, PAIR);
-                ok = bar_and(BAR_SOFT, NSOFT, done);
+            bool ok;
+            {
+                bool done = false;
+                if (!err) done = wait_bar(o_done, (nT - 1) & 1, wc, SITE_O_DONE, true, PAIR);
+                ok = bar_and(BAR_SOFT, NSOFT, done);  // reached by all 256 threads
             }
             if (ok) {
                 tc_fence_after();
