@@ -101,19 +101,23 @@ struct Cfg {
     static constexpr uint32_t OFF_V = OFF_K + NK * KST_BYTES;
     static constexpr uint32_t OFF_BAR = OFF_V + NV * VST_BYTES;
     // q_full, k_full[NK], k_empty[NK], v_full[NV], v_ready[NV], v_empty[NV],
-    // s_full[2], p_full[2], o_done, drain
-    static constexpr int NBAR = 1 + 2 * NK + 3 * NV + 2 + 2 + 1 + 1;
+    // s_full[2], p_full[2], pd_full[2], o_done, drain
+    static constexpr int NBAR = 1 + 2 * NK + 3 * NV + 2 + 2 + 2 + 1 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t OFF_XCH = OFF_MISC + 16;  // float [2][2][128]
     static constexpr uint32_t SMEM_BYTES = OFF_XCH + 2 * 2 * 128 * 4;
-    // TMEM columns: O | O'_acc | S buffer 0 (S, S'_raw) | S buffer 1.  Inside an S
-    // buffer, bf16 P goes to columns [16, 48) and P (sS' - c) to [80, 112):
-    // each softmax warpgroup then overwrites only columns it has read itself.
+    // TMEM columns: O | O'_acc | S buffer 0 (S, S'_raw) | S buffer 1.  Both
+    // softmax warpgroups read all of S (the row max) but only their own half
+    // of S'_raw, columns [BN + 32g, BN + 32g + 32).  Warpgroup g writes its
+    // bf16 P (keys 32g..32g+31, two per column) over the first 16 of those
+    // columns and P (sS' - c) over the last 16, so no one overwrites a
+    // column another warp may still read.
     static constexpr uint32_t T_O = 0;
     static constexpr uint32_t T_OD = D;
     static constexpr uint32_t T_S = 2 * D;
-    static constexpr uint32_t T_P = 16;        // offset of bf16 P inside an S buffer
-    static constexpr uint32_t T_PD = BN + 16;  // offset of bf16 P (sS' - c)
+    // column of the bf16 P (pd = false) or P (sS' - c) (pd = true) operand of
+    // keys 16kk..16kk+15 inside an S buffer
+    __host__ __device__ static constexpr uint32_t t_pk(int kk, bool pd) { return BN + (kk >> 1) * 32 + (pd ? 16 : 0) + (kk & 1) * 8; }
     static constexpr int MMA_M = BM * NCTA;
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(MMA_M, 2 * BN, false);
     static constexpr uint32_t IDESC_SD = idesc_bf16_f32(MMA_M, BN, false);
@@ -250,8 +254,9 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
     uint64_t *v_ready = v_full + C::NV;
     uint64_t *v_empty = v_ready + C::NV;
     uint64_t *s_full = v_empty + C::NV;
-    uint64_t *p_full = s_full + 2;
-    uint64_t *o_done = p_full + 2;
+    uint64_t *p_full = s_full + 2;   // [2] bf16 P written
+    uint64_t *pd_full = p_full + 2;  // [2] bf16 P (sS' - c) written
+    uint64_t *o_done = pd_full + 2;
     uint64_t *drain = o_done + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
@@ -270,6 +275,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], C::P_ARRIVALS);
+            mbar_init(&pd_full[s], C::P_ARRIVALS);
         }
         mbar_init(o_done, 1);
         mbar_init(drain, 1);
@@ -308,8 +314,10 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
     const uint32_t k_full_lead = PAIR ? mapa_shared(smem_addr(k_full), 0) : smem_addr(k_full);
     const uint32_t v_ready_lead = PAIR ? mapa_shared(smem_addr(v_ready), 0) : smem_addr(v_ready);
     const uint32_t p_full_lead = PAIR ? mapa_shared(smem_addr(p_full), 0) : smem_addr(p_full);
+    const uint32_t pd_full_lead = PAIR ? mapa_shared(smem_addr(pd_full), 0) : smem_addr(pd_full);
     (void)v_ready_lead;
     (void)p_full_lead;
+    (void)pd_full_lead;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -423,131 +431,125 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
             // addresses fit its 18 bits), which keeps the issue loop short.
             const uint64_t dq = sdesc_sw128(smem_addr(smem + C::OFF_Q), 16, 1024);
             const uint64_t dqd = sdesc_sw128(smem_addr(smem + C::OFF_QD), 16, 1024);
-            // S_js and PV_jp are issued in whichever order their inputs arrive,
-            // with S at most one tile ahead of PV (S_js overwrites the buffer
-            // that held P_{js-2}, so PV_{js-2} must already be issued).  A late
-            // K tile then never holds back a PV whose P is ready.
-            // The wait limit runs from the first idle check after the last
-            // issue: reading %globaltimer costs hundreds of clocks, so the
-            // issue path never reads it.
-            int js = 0, jp = 0, polls = 0;
-            bool idle_timed = false;
-            uint64_t t_idle = 0;
-            auto test = [&](uint64_t *bar, uint32_t parity) {
-                return __all_sync(0xffffffffu, PAIR ? mbar_test_wait_cluster(smem_addr(bar), parity)
-                                                    : mbar_test_wait(smem_addr(bar), parity));
+            // Fixed order S_0, S_1, PV_0, S_2, PV_1, ...: S_{j+1} runs on the
+            // tensor core while the softmax works on tile j, and S_{j+1}
+            // overwrites the TMEM buffer that held P_{j-1} only after PV_{j-1}
+            // was issued (MMAs run in issue order).  Each wait first parks the
+            // warp in mbarrier.try_wait, which wakes it when the phase completes.
+            auto wait_u = [&](uint64_t *bar, uint32_t parity, int site) {
+                const uint32_t a = smem_addr(bar);
+                bool r = PAIR ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity);
+                if (!__all_sync(0xffffffffu, r)) r = wait_bar(bar, parity, wc, site, true, PAIR);
+                return __all_sync(0xffffffffu, r);
             };
-            while (ok && jp < nT) {
-                bool progressed = false;
-                if (js < nT && js <= jp + 1 && test(&k_full[js % C::NK], (js / C::NK) & 1)) {
-                    const int j = js;
-                    const int s = j % C::NK;
-                    tc_fence_after();
-                    const uint32_t tS = tbase + C::T_S + (j & 1) * (2 * BN);
-                    const uint64_t dk = sdesc_sw128(smem_addr(smem + C::OFF_K + s * C::KST_BYTES), 16, 1024);
-                    if constexpr (PAIR) {
-                        // S | Q K'^T = Q [K ; K']^T: B rows 0-63 (K) in the leader, 64-127 (K') in the peer
+            auto issue_s = [&](const int j) {
+                const int s = j % C::NK;
+                tc_fence_after();
+                const uint32_t tS = tbase + C::T_S + (j & 1) * (2 * BN);
+                const uint64_t dk = sdesc_sw128(smem_addr(smem + C::OFF_K + s * C::KST_BYTES), 16, 1024);
+                if constexpr (PAIR) {
+                    // S | Q K'^T = Q [K ; K']^T: B rows 0-63 (K) in the leader, 64-127 (K') in the peer
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                            const uint32_t ob = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-                            mma_ss_pair(tS, desc_add(dq, oa), desc_add(dk, ob),
-                                        C::IDESC_S, kk > 0 ? 1u : 0u);
-                        }
-                        // += Q' K^T: B rows 0-31 of K in the leader, 32-63 in the peer
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                            const uint32_t ob = C::X_BYTES + (kk >> 2) * (BN / 2 * 128) + (kk & 3) * 32;
-                            mma_ss_pair(tS + BN, desc_add(dqd, oa), desc_add(dk, ob),
-                                        C::IDESC_SD, 1u);
-                        }
-                        mma_commit_pair_mc(&k_empty[s], 0x3);
-                        mma_commit_pair_mc(&s_full[j & 1], 0x3);
-                    } else {
-                        // S | Q K'^T  =  Q [K ; K']^T   (N = 2 BN)
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                            const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
-                            mma_ss(tS, desc_add(dq, oa), desc_add(dk, ob),
-                                   C::IDESC_S, kk > 0 ? 1u : 0u);
-                        }
-                        // += Q' K^T into the second half
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                            const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
-                            mma_ss(tS + BN, desc_add(dqd, oa), desc_add(dk, ob),
-                                   C::IDESC_SD, 1u);
-                        }
-                        mma_commit(&k_empty[s]);
-                        mma_commit(&s_full[j & 1]);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        const uint32_t ob = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+                        mma_ss_pair(tS, desc_add(dq, oa), desc_add(dk, ob),
+                                    C::IDESC_S, kk > 0 ? 1u : 0u);
                     }
-                    issued = true;
-                    ++js;
-                    progressed = true;
-                } else if (jp < js && test(&p_full[jp & 1], (jp >> 1) & 1) &&
-                           test(PAIR ? &v_ready[jp % C::NV] : &v_full[jp % C::NV], (jp / C::NV) & 1)) {
-                    const int jj = jp;
-                    const int s = jj % C::NV;
-                    tc_fence_after();
-                    const uint32_t tP = tbase + C::T_S + (jj & 1) * (2 * BN);
-                    // LBO: distance between 64-column blocks of V (single CTA, d = 128);
-                    // a pair CTA holds one block, so it is unused there
-                    constexpr uint32_t LBO = BN * 128;
-                    const uint64_t dv = sdesc_sw128(smem_addr(smem + C::OFF_V + s * C::VST_BYTES), LBO, 1024);
-                    const uint64_t dvd = desc_add(dv, C::VHALF_BYTES);
+                    // += Q' K^T: B rows 0-31 of K in the leader, 32-63 in the peer
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {  // O += P V
-                        const uint32_t a = tP + C::T_P + kk * 8;
-                        const uint64_t bd = desc_add(dv, kk * 2048);
-                        const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
-                        if constexpr (PAIR) mma_ts_pair(tbase + C::T_O, a, bd, C::IDESC_PV, acc);
-                        else mma_ts(tbase + C::T_O, a, bd, C::IDESC_PV, acc);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        const uint32_t ob = C::X_BYTES + (kk >> 2) * (BN / 2 * 128) + (kk & 3) * 32;
+                        mma_ss_pair(tS + BN, desc_add(dqd, oa), desc_add(dk, ob),
+                                    C::IDESC_SD, 1u);
                     }
+                    mma_commit_pair_mc(&k_empty[s], 0x3);
+                    mma_commit_pair_mc(&s_full[j & 1], 0x3);
+                } else {
+                    // S | Q K'^T  =  Q [K ; K']^T   (N = 2 BN)
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P(sS' - c) V
-                        const uint32_t a = tP + C::T_PD + kk * 8;
-                        const uint64_t bd = desc_add(dv, kk * 2048);
-                        const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
-                        if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, bd, C::IDESC_PV, acc);
-                        else mma_ts(tbase + C::T_OD, a, bd, C::IDESC_PV, acc);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
+                        mma_ss(tS, desc_add(dq, oa), desc_add(dk, ob),
+                               C::IDESC_S, kk > 0 ? 1u : 0u);
                     }
+                    // += Q' K^T into the second half
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P V'
-                        const uint32_t a = tP + C::T_P + kk * 8;
-                        const uint64_t bd = desc_add(dvd, kk * 2048);
-                        if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, bd, C::IDESC_PV, 1u);
-                        else mma_ts(tbase + C::T_OD, a, bd, C::IDESC_PV, 1u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
+                        mma_ss(tS + BN, desc_add(dqd, oa), desc_add(dk, ob),
+                               C::IDESC_SD, 1u);
                     }
-                    if constexpr (PAIR) {
-                        mma_commit_pair_mc(&v_empty[s], 0x3);
-                        mma_commit_pair_mc(o_done, 0x3);
-                    } else {
-                        mma_commit(&v_empty[s]);
-                        mma_commit(o_done);
-                    }
-                    ++jp;
-                    progressed = true;
+                    mma_commit(&k_empty[s]);
+                    mma_commit(&s_full[j & 1]);
                 }
-                if (progressed) {
-                    polls = 0;
-                    idle_timed = false;
-                } else if (++polls >= 64) {
-                    polls = 0;
-                    const uint64_t now = __shfl_sync(0xffffffffu, globaltimer_ns(), 0);
-                    if (__any_sync(0xffffffffu, *abort_flag != 0)) {
-                        ok = false;
-                    } else if (!idle_timed) {
-                        idle_timed = true;
-                        t_idle = now;
-                    } else if (now - t_idle > p.timeout_ns) {
-                        *abort_flag = 1;
-                        atomicCAS(&g_status, 0, js < nT && js <= jp + 1 ? SITE_K_FULL : SITE_P_FULL);
-                        ok = false;
-                    }
+                issued = true;
+            };
+            // LBO: distance between 64-column blocks of V (single CTA, d = 128);
+            // a pair CTA holds one block, so it is unused there
+            constexpr uint32_t LBO = BN * 128;
+            // PV_j in two groups: A needs only P (O += P V, O'_acc += P V'),
+            // B needs P (sS' - c) as well (O'_acc += P (sS' - c) V), which the
+            // softmax writes later; A can then start while B's operand is formed.
+            auto issue_pa = [&](const int jj) {
+                const int s = jj % C::NV;
+                tc_fence_after();
+                const uint32_t tP = tbase + C::T_S + (jj & 1) * (2 * BN);
+                const uint64_t dv = sdesc_sw128(smem_addr(smem + C::OFF_V + s * C::VST_BYTES), LBO, 1024);
+                const uint64_t dvd = desc_add(dv, C::VHALF_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {  // O += P V
+                    const uint32_t a = tP + C::t_pk(kk, false);
+                    const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+                    if constexpr (PAIR) mma_ts_pair(tbase + C::T_O, a, desc_add(dv, kk * 2048), C::IDESC_PV, acc);
+                    else mma_ts(tbase + C::T_O, a, desc_add(dv, kk * 2048), C::IDESC_PV, acc);
                 }
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P V'
+                    const uint32_t a = tP + C::t_pk(kk, false);
+                    const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+                    if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, desc_add(dvd, kk * 2048), C::IDESC_PV, acc);
+                    else mma_ts(tbase + C::T_OD, a, desc_add(dvd, kk * 2048), C::IDESC_PV, acc);
+                }
+            };
+            auto issue_pb = [&](const int jj) {
+                const int s = jj % C::NV;
+                tc_fence_after();
+                const uint32_t tP = tbase + C::T_S + (jj & 1) * (2 * BN);
+                const uint64_t dv = sdesc_sw128(smem_addr(smem + C::OFF_V + s * C::VST_BYTES), LBO, 1024);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P(sS' - c) V
+                    const uint32_t a = tP + C::t_pk(kk, true);
+                    if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, desc_add(dv, kk * 2048), C::IDESC_PV, 1u);
+                    else mma_ts(tbase + C::T_OD, a, desc_add(dv, kk * 2048), C::IDESC_PV, 1u);
+                }
+                if constexpr (PAIR) {
+                    mma_commit_pair_mc(&v_empty[s], 0x3);
+                    mma_commit_pair_mc(o_done, 0x3);
+                } else {
+                    mma_commit(&v_empty[s]);
+                    mma_commit(o_done);
+                }
+            };
+            if (ok) ok = wait_u(&k_full[0], 0, SITE_K_FULL);
+            if (ok) issue_s(0);
+            for (int j = 0; ok && j < nT; ++j) {
+                if (j + 1 < nT) {
+                    ok = wait_u(&k_full[(j + 1) % C::NK], ((j + 1) / C::NK) & 1, SITE_K_FULL);
+                    if (!ok) break;
+                    issue_s(j + 1);
+                }
+                // V_j normally lands before P_j is written: wait for it first
+                ok = wait_u(PAIR ? &v_ready[j % C::NV] : &v_full[j % C::NV], (j / C::NV) & 1, SITE_V_FULL);
+                if (ok) ok = wait_u(&p_full[j & 1], (j >> 1) & 1, SITE_P_FULL);
+                if (!ok) break;
+                issue_pa(j);
+                ok = wait_u(&pd_full[j & 1], (j >> 1) & 1, SITE_P_FULL);
+                if (!ok) break;
+                issue_pb(j);
             }
             if (!ok && issued) {
                 if constexpr (PAIR) mma_commit_pair_mc(drain, 0x1);
@@ -626,6 +628,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                 const uint32_t tS = tbase + lane_off + C::T_S + bsel * (2 * BN);
                 if (!__all_sync(0xffffffffu, wait_bar_fast(&s_full[bsel], (j >> 1) & 1, wc, SITE_S_FULL, PAIR))) {
                     err = true;
+                    if (j == 0) bar_and(BAR_SOFT, NSOFT, false);  // the others wait there at tile 0
                     break;
                 }
                 tc_fence_after();
@@ -698,70 +701,28 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                 if (j == 0) {
                     // centring constant c: the p-weighted mean of s S' over the
                     // first 32 keys (warpgroup 0's half, which always holds a
-                    // valid key).  Warpgroup 1 forms the same p from the same S
-                    // bits with the same instructions, so both get the same c.
-                    float pc[32], dc[32];
+                    // valid key), handed to warpgroup 1 through shared memory
                     if (g == 0) {
+                        float n0 = 0.f, n1 = 0.f, w0 = 0.f, w1 = 0.f;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            pc[i] = x[i];
-                            dc[i] = u2f(rd[i]);
+                        for (int i = 0; i < 32; i += 2) {
+                            n0 += (tail && i >= valid) ? 0.f : x[i] * (u2f(rd[i]) * sc);
+                            n1 += (tail && i + 1 >= valid) ? 0.f : x[i + 1] * (u2f(rd[i + 1]) * sc);
+                            w0 += x[i];
+                            w1 += x[i + 1];
                         }
-                    } else {
-                        uint32_t cs[32], cdr[32];
-                        tmem_ld32(tS, cs);
-                        tmem_ld32(tS + BN, cdr);
-                        tmem_ld_wait2(cs, cdr);
-                        const uint64_t sl22 = f2_pack(sl2, sl2);
-                        const uint64_t nm2 = f2_pack(-m_used, -m_used);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float t0, t1;
-                            f2_unpack(f2_fma(f2_pack(u2f(cs[2 * i]), u2f(cs[2 * i + 1])), sl22, nm2), t0, t1);
-                            pc[2 * i] = (2 * i < vt) ? ex2_approx(t0) : 0.f;
-                            pc[2 * i + 1] = (2 * i + 1 < vt) ? ex2_approx(t1) : 0.f;
-                        }
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) dc[i] = u2f(cdr[i]);
+                        cctr = (n0 + n1) / (w0 + w1);
+                        xch[r] = cctr;
                     }
-                    float n0 = 0.f, n1 = 0.f, w0 = 0.f, w1 = 0.f;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        n0 = (i >= vt) ? n0 : __fmaf_rn(pc[i], __fmul_rn(dc[i], sc), n0);
-                        n1 = (i + 1 >= vt) ? n1 : __fmaf_rn(pc[i + 1], __fmul_rn(dc[i + 1], sc), n1);
-                        w0 = __fadd_rn(w0, pc[i]);
-                        w1 = __fadd_rn(w1, pc[i + 1]);
+                    if (!bar_and(BAR_SOFT, NSOFT, true)) {
+                        err = true;
+                        break;
                     }
-                    cctr = __fdiv_rn(__fadd_rn(n0, n1), __fadd_rn(w0, w1));
+                    if (g == 1) cctr = xch[r];
                 }
-                // bf16 operands of the PV MMAs: P and P (s S' - c)
-                uint32_t pk[16], pdk[16];
-                {
-                    const uint64_t sc2 = f2_pack(sc, sc);
-                    const uint64_t nc2 = f2_pack(-cctr, -cctr);
-                    uint64_t a0 = 0, a1 = 0;
+                uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint64_t p2 = f2_pack(x[2 * i], x[2 * i + 1]);
-                        const uint64_t d2 = f2_mul(f2_fma(f2_pack(u2f(rd[2 * i]), u2f(rd[2 * i + 1])), sc2, nc2), p2);
-                        float d0, d1;
-                        f2_unpack(d2, d0, d1);
-                        if (tail) {
-                            d0 = (2 * i < valid) ? d0 : 0.f;
-                            d1 = (2 * i + 1 < valid) ? d1 : 0.f;
-                        }
-                        pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-                        pdk[i] = pack_bf16x2(d0, d1);
-                        // the two rounded values as fp32
-                        const uint64_t r2 = f2_pack(u2f(pdk[i] << 16), u2f(pdk[i] & 0xFFFF0000u));
-                        if (i & 1) a1 = f2_add(a1, r2);
-                        else a0 = f2_add(a0, r2);
-                    }
-                    float u0, u1, u2, u3;
-                    f2_unpack(a0, u0, u1);
-                    f2_unpack(a1, u2, u3);
-                    acc_a += (u0 + u1) + (u2 + u3);
-                }
+                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
                 if (j >= 1) {
                     // PV of the previous tile must be done before O may be
                     // rescaled; every warp observes every phase of o_done in
@@ -806,14 +767,49 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                     }
                     fence_proxy_async_smem();
                 }
-                tmem_st16(tS + C::T_P + 16 * g, pk);
-                tmem_st16(tS + C::T_PD + 16 * g, pdk);
+                // P over the first 16 columns of this half of S'_raw (read above)
+                tmem_st16(tS + BN + c0, pk);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
                     if constexpr (PAIR) mbar_arrive_cluster(p_full_lead + bsel * 8);
                     else mbar_arrive(&p_full[bsel]);
+                }
+                // ---- bf16 P (s S' - c) while the tensor core multiplies P
+                uint32_t pdk[16];
+                {
+                    const uint64_t sc2 = f2_pack(sc, sc);
+                    const uint64_t nc2 = f2_pack(-cctr, -cctr);
+                    uint64_t a0 = 0, a1 = 0;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const uint64_t p2 = f2_pack(x[2 * i], x[2 * i + 1]);
+                        const uint64_t d2 = f2_mul(f2_fma(f2_pack(u2f(rd[2 * i]), u2f(rd[2 * i + 1])), sc2, nc2), p2);
+                        float d0, d1;
+                        f2_unpack(d2, d0, d1);
+                        if (tail) {
+                            d0 = (2 * i < valid) ? d0 : 0.f;
+                            d1 = (2 * i + 1 < valid) ? d1 : 0.f;
+                        }
+                        pdk[i] = pack_bf16x2(d0, d1);
+                        // the two rounded values as fp32
+                        const uint64_t r2 = f2_pack(u2f(pdk[i] << 16), u2f(pdk[i] & 0xFFFF0000u));
+                        if (i & 1) a1 = f2_add(a1, r2);
+                        else a0 = f2_add(a0, r2);
+                    }
+                    float u0, u1, u2, u3;
+                    f2_unpack(a0, u0, u1);
+                    f2_unpack(a1, u2, u3);
+                    acc_a += (u0 + u1) + (u2 + u3);
+                }
+                tmem_st16(tS + BN + c0 + 16, pdk);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (PAIR) mbar_arrive_cluster(pd_full_lead + bsel * 8);
+                    else mbar_arrive(&pd_full[bsel]);
                 }
             }
             bool ok;
