@@ -69,13 +69,21 @@ def kernel_source_hash() -> str:
 
 
 def load_peaks():
+    """(burst bf16 TFLOP/s, sustained bf16 TFLOP/s or None, HBM GB/s, source)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             pk = json.load(f)
-        return float(pk["bf16_tflops"]), float(pk["hbm_gbs"]), "measured"
+        sus = pk.get("bf16_tflops_sustained")
+        return (float(pk["bf16_tflops"]), float(sus) if sus else None, float(pk["hbm_gbs"]),
+                "measured")
     except (OSError, KeyError, ValueError):
-        return FALLBACK_PEAKS["bf16_tflops"], FALLBACK_PEAKS["hbm_gbs"], "fallback"
+        return FALLBACK_PEAKS["bf16_tflops"], None, FALLBACK_PEAKS["hbm_gbs"], "fallback"
+
+
+# A timed region this long runs the GPU into its power cap, like the
+# seconds-long cuBLAS loop behind the sustained peak.
+SUSTAINED_MS = 500.0
 
 
 def measured_traffic(workload: str):
@@ -380,7 +388,11 @@ def run_ours(args):
     h2d = in_bytes
     d2h = (o.numel() + od.numel()) * 2 + lse.numel() * 4
 
-    peak_tf, peak_hbm, peak_src = load_peaks()
+    burst_tf, sustained_tf, peak_hbm, peak_src = load_peaks()
+    if sustained_tf is not None and local_ms >= SUSTAINED_MS:
+        peak_tf, peak_kind = sustained_tf, "sustained"
+    else:
+        peak_tf, peak_kind = burst_tf, "burst"
     per_launch_ms = local_ms / args.steps
     achieved = flops_step / (per_launch_ms * 1e-3) / 1e12
     traffic = measured_traffic(args.workload)
@@ -391,8 +403,10 @@ def run_ours(args):
         "config": workload_config(w, args),
         "gpu_launches": args.steps,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf,
-                     "peak_source": f"{peak_src} bf16 dense (burst)", "unit": UNIT,
-                     "frac": achieved / peak_tf, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 dense ({peak_kind}; timed region "
+                                    f"{local_ms:.0f} ms)", "unit": UNIT,
+                     "frac": achieved / peak_tf, "frac_of_burst_peak": achieved / burst_tf,
+                     "traffic": traffic,
                      "algorithmic_bytes": algorithmic_bytes(w),
                      "flops_per_launch": flops_step,
                      "kernel": f"attn_jvp_fwd_kernel<{d}>"},
