@@ -59,7 +59,7 @@ def _bind(lib):
     f.restype = ctypes.c_int
     f.argtypes = ([ctypes.c_int] + [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5
                   + [ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64]
-                  + [ctypes.c_void_p] * 3 + [ctypes.c_int])
+                  + [ctypes.c_void_p] * 4 + [ctypes.c_int])
     lib.oracle_max_threads.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     return lib
@@ -74,7 +74,7 @@ def _ptr(a: np.ndarray) -> int:
 
 
 def attn_jvp(q, k, v, q_dot, k_dot, v_dot, scale, kv_len=None, rows=None,
-             n_threads: int = 0, lib=None):
+             n_threads: int = 0, lib=None, lse_dot: bool = False):
     """Run the oracle.
 
     Inputs are either ``uint16`` arrays of bf16 bit patterns or ``float64``
@@ -83,7 +83,8 @@ def attn_jvp(q, k, v, q_dot, k_dot, v_dot, scale, kv_len=None, rows=None,
     selects flat query rows ``(b*H + h)*Lq + i``; the outputs then have a
     leading dimension ``len(rows)`` instead of ``[B, H, Lq]``.
 
-    Returns ``(o, o_dot, lse)`` in float64.
+    Returns ``(o, o_dot, lse)`` in float64, and ``lse_dot`` (the tangent of
+    lse, mu = sum_j P S') as a fourth array when ``lse_dot`` is set.
     """
     lib = lib or load_library()
     arrs = [q, k, v, q_dot, k_dot, v_dot]
@@ -116,11 +117,12 @@ def attn_jvp(q, k, v, q_dot, k_dot, v_dot, scale, kv_len=None, rows=None,
     o = np.empty(out_shape + (d,), np.float64)
     od = np.empty(out_shape + (d,), np.float64)
     lse = np.empty(out_shape, np.float64)
+    mu = np.empty(out_shape, np.float64) if lse_dot else None
     if rows is not None and nr == 0:
-        return o, od, lse
+        return (o, od, lse, mu) if lse_dot else (o, od, lse)
     rc = lib.oracle_attn_jvp(dtype, *[_ptr(a) for a in arrs], B, H, Lq, Lk, d,
                              float(scale), kvp, rp, nr, _ptr(o), _ptr(od), _ptr(lse),
-                             int(n_threads))
+                             _ptr(mu) if lse_dot else None, int(n_threads))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_jvp failed with code {rc}")
-    return o, od, lse
+    return (o, od, lse, mu) if lse_dot else (o, od, lse)

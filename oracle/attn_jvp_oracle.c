@@ -23,16 +23,19 @@
  *   O'_i   = sum_j P_ij (S'_ij - mu_i) v_j + sum_j P_ij v'_j
  *
  * (P' = P (S' - mu) is the derivative of the row softmax; O' = P' V + P V'.)
+ * mu_i is also the tangent of lse_i (d lse = sum_j P_ij dS_ij) and is
+ * returned as lse' when asked for.
  *
  * Readings where the pages say nothing:
  *   - n_b = min(Lk, kv_len[b]) clamped at 0; kv_len == NULL means n_b = Lk.
  *     Keys j >= n_b take no part: their k, k', v, v' are never read.
- *   - n_b == 0: O = O' = 0 and lse = -inf.
+ *   - n_b == 0: O = O' = 0, lse = -inf and lse' = 0 (a constant has no
+ *     tangent).
  *   - lse is the natural logarithm, in units of the scaled logits.
  *   - Inputs are either bf16 bit patterns (widened exactly to fp64) or fp64.
  *
  * Layout: q, q', o, o' are [B, H, Lq, d]; k, k', v, v' are [B, H, Lk, d];
- * lse is [B, H, Lq]; all dense row-major.  With a row subset, output r holds
+ * lse and lse' are [B, H, Lq]; all dense row-major.  With a row subset, output r holds
  * flat query row rows[r] (row = (b*H + h)*Lq + i).
  *
  * Built with -O2 -ffp-contract=off and no fast-math, so every sum is the
@@ -81,7 +84,7 @@ static double dot(const double *a, const double *b, int d)
 static void one_row(int dtype, const void *q, const void *k, const void *v,
                     const void *qd, const void *kd, const void *vd,
                     int H, int Lq, int Lk, int d, double scale, const int32_t *kv_len,
-                    int64_t row, double *o, double *od, double *lse,
+                    int64_t row, double *o, double *od, double *lse, double *lse_dot,
                     double *S, double *P, double *Sd, double *qi, double *qdi,
                     double *kj, double *kdj, double *vj, double *vdj)
 {
@@ -97,6 +100,7 @@ static void one_row(int dtype, const void *q, const void *k, const void *v,
     if (n == 0) {
         for (int c = 0; c < d; ++c) { o[c] = 0.0; od[c] = 0.0; }
         *lse = -INFINITY;
+        if (lse_dot) *lse_dot = 0.0;
         return;
     }
     size_t qoff = (size_t)(bh * Lq + i) * (size_t)d;
@@ -123,6 +127,7 @@ static void one_row(int dtype, const void *q, const void *k, const void *v,
     /* mu = sum_j P_j S'_j */
     double mu = 0.0;
     for (int j = 0; j < n; ++j) mu += P[j] * Sd[j];
+    if (lse_dot) *lse_dot = mu;
 
     /* O = P V ;  O' = sum_j P_j (S'_j - mu) v_j + sum_j P_j v'_j */
     for (int c = 0; c < d; ++c) { o[c] = 0.0; od[c] = 0.0; }
@@ -147,13 +152,14 @@ static void one_row(int dtype, const void *q, const void *k, const void *v,
 
 /*
  * Returns 0 on success, -1 on a bad argument, -2 if scratch could not be
- * allocated.  n_threads <= 0 lets OpenMP choose.
+ * allocated.  lse_dot may be NULL (not computed).  n_threads <= 0 lets OpenMP
+ * choose.
  */
 int oracle_attn_jvp(int dtype, const void *q, const void *k, const void *v,
                     const void *qd, const void *kd, const void *vd,
                     int B, int H, int Lq, int Lk, int d, double scale,
                     const int32_t *kv_len, const int64_t *rows, int64_t n_rows,
-                    double *o, double *od, double *lse, int n_threads)
+                    double *o, double *od, double *lse, double *lse_dot, int n_threads)
 {
     if (!q || !k || !v || !qd || !kd || !vd || !o || !od || !lse) return -1;
     if (B < 1 || H < 1 || Lq < 1 || Lk < 1 || d < 1) return -1;
@@ -186,7 +192,7 @@ int oracle_attn_jvp(int dtype, const void *q, const void *k, const void *v,
         double *rb = Sd + Lk;
         int64_t row = rows ? rows[r] : r;
         one_row(dtype, q, k, v, qd, kd, vd, H, Lq, Lk, d, scale, kv_len, row,
-                o + (size_t)r * d, od + (size_t)r * d, lse + r, S, P, Sd,
+                o + (size_t)r * d, od + (size_t)r * d, lse + r, lse_dot ? lse_dot + r : NULL, S, P, Sd,
                 rb, rb + d, rb + 2 * d, rb + 3 * d, rb + 4 * d, rb + 5 * d);
     }
     free(scratch);

@@ -297,7 +297,65 @@ def pin_hand_examples(lib):
         assert np.allclose(lse[fin], el[fin], rtol=1e-14, atol=1e-14), c["name"]
 
 
+def run_mu(lib, q, k, v, qd, kd, vd, scale, kv_len=None, rows=None):
+    return oracle.attn_jvp(q, k, v, qd, kd, vd, scale, kv_len=kv_len, rows=rows,
+                           lib=lib, n_threads=2, lse_dot=True)
+
+
+def pin_lse_dot_finite_difference(lib):
+    """lse' against (lse(x + eps x') - lse(x - eps x')) / (2 eps), eps = 1e-6,
+    for Q' and K' alone and together; V' must not move it."""
+    q, k, v, qd, kd, vd = _rand(23, 1, 2, 5, 7, 4)
+    s = 0.9
+    eps = 1e-6
+    z = np.zeros_like
+    for tq, tk in [(qd, kd), (qd, z(kd)), (z(qd), kd)]:
+        _, _, _, mu = run_mu(lib, q, k, v, tq, tk, vd, s)
+        _, _, lp = run(lib, q + eps * tq, k + eps * tk, v, tq, tk, vd, s)
+        _, _, lm = run(lib, q - eps * tq, k - eps * tk, v, tq, tk, vd, s)
+        fd = (lp - lm) / (2 * eps)
+        assert rel(mu, fd) < 1e-7, f"lse' finite difference mismatch {rel(mu, fd)}"
+        _, _, _, mu0 = run_mu(lib, q, k, v, tq, tk, z(vd), s)
+        assert np.array_equal(mu, mu0), "V' changed lse'"
+
+
+def pin_lse_dot_torch_jvp(lib):
+    """lse' against torch.func.jvp of torch.logsumexp over plain fp64 logits."""
+    q, k, v, qd, kd, vd = _rand(29, 2, 2, 6, 9, 8)
+    s = 0.35
+    _, _, _, mu = run_mu(lib, q, k, v, qd, kd, vd, s)
+    f = lambda qq, kk: torch.logsumexp(s * qq @ kk.transpose(-1, -2), dim=-1)
+    _, ref = torch.func.jvp(f, (torch.from_numpy(q), torch.from_numpy(k)),
+                            (torch.from_numpy(qd), torch.from_numpy(kd)))
+    assert rel(mu, ref.numpy()) < 1e-12, f"lse' vs torch.func.jvp {rel(mu, ref.numpy())}"
+
+
+def pin_lse_dot_closed_forms(lib):
+    """One key: lse' = s (q'.k + q.k').  Equal keys with K' = 0: lse' = s q'.k.
+    No valid key: lse' = 0.  Padded keys (NaN) do not reach it."""
+    q, k, v, qd, kd, vd = _rand(31, 1, 1, 4, 1, 5)
+    s = 1.3
+    _, _, _, mu = run_mu(lib, q, k, v, qd, kd, vd, s)
+    ref = s * (np.einsum("bhid,bhd->bhi", qd, k[:, :, 0]) + np.einsum("bhid,bhd->bhi", q, kd[:, :, 0]))
+    assert rel(mu, ref) < 1e-13, "single-key lse'"
+    q, k, v, qd, kd, vd = _rand(37, 1, 1, 3, 6, 4)
+    k[:] = k[:, :, :1]
+    _, _, _, mu = run_mu(lib, q, k, v, qd, np.zeros_like(kd), vd, s)
+    ref = s * np.einsum("bhid,bhd->bhi", qd, k[:, :, 0])
+    assert rel(mu, ref) < 1e-13, "equal-keys lse'"
+    q, k, v, qd, kd, vd = _rand(41, 2, 1, 3, 8, 4)
+    kv = np.array([0, 5], np.int32)
+    _, _, _, mu = run_mu(lib, q, k, v, qd, kd, vd, s, kv_len=kv)
+    assert np.all(mu[0] == 0.0), "lse' of a row without keys"
+    k2, kd2 = k.copy(), kd.copy()
+    k2[1, :, 5:] = np.nan
+    kd2[1, :, 5:] = np.nan
+    _, _, _, mu2 = run_mu(lib, q, k2, v, qd, kd2, vd, s, kv_len=kv)
+    assert np.array_equal(mu[1], mu2[1]), "padded keys reached lse'"
+
+
 PINS = [pin_finite_difference, pin_torch_jvp, pin_explicit_jacobian, pin_vdot_equals_v,
         pin_equal_keys, pin_linearity, pin_single_key, pin_zero_scale, pin_equal_values,
         pin_key_permutation, pin_masking, pin_large_logits, pin_row_subset,
-        pin_bf16_inputs, pin_hand_examples]
+        pin_bf16_inputs, pin_hand_examples, pin_lse_dot_finite_difference,
+        pin_lse_dot_torch_jvp, pin_lse_dot_closed_forms]

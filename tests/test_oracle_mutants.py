@@ -32,6 +32,8 @@ MUTANTS = [
     ("mask_off_by_one", "n = kv_len[b];", "n = kv_len[b] + 1;"),
     ("value_row_index", "for (int c = 0; c < d; ++c) o[c] += P[j] * vj[c];",
      "for (int c = 0; c < d; ++c) o[c] += P[j] * vj[(c + 1) % d];"),
+    ("lse_dot_sign", "if (lse_dot) *lse_dot = mu;", "if (lse_dot) *lse_dot = -mu;"),
+    ("lse_dot_unnormalised", "if (lse_dot) *lse_dot = mu;", "if (lse_dot) *lse_dot = mu * l;"),
     ("query_tangent_row", "widen_row(qd, dtype, qoff, d, qdi);",
      "widen_row(qd, dtype, qoff - (i > 0 ? d : 0), d, qdi);"),
 ]
