@@ -26,8 +26,8 @@ ATTN_JVP_ERR_VALUE = -7
 ATTN_JVP_DEBUG_STARVE_Q = 1
 ATTN_JVP_DEBUG_CTA_PAIR = 2
 
-EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_debug", "attn_jvp_check", "attn_jvp_status_string",
-            "attn_jvp_version")
+EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_ex", "attn_jvp_fwd_debug", "attn_jvp_check",
+            "attn_jvp_status_string", "attn_jvp_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -57,6 +57,8 @@ def load_library():
             vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
             lib.attn_jvp_fwd.restype = i32
             lib.attn_jvp_fwd.argtypes = [vp] * 9 + [i32] * 5 + [f32, vp, vp]
+            lib.attn_jvp_fwd_ex.restype = i32
+            lib.attn_jvp_fwd_ex.argtypes = [vp] * 10 + [i32] * 5 + [f32, vp, vp]
             lib.attn_jvp_fwd_debug.restype = i32
             lib.attn_jvp_fwd_debug.argtypes = [vp] * 9 + [i32] * 5 + [f32, vp, vp,
                                                                      ctypes.c_uint64, i32]
@@ -75,8 +77,12 @@ def attn_jvp_status_string(status: int) -> str:
 
 
 def _check_inputs(q, k, v, q_dot, k_dot, v_dot):
+    if (k_dot is None) != (v_dot is None):
+        raise ValueError("k_dot and v_dot must both be tensors or both be None (K' = V' = 0)")
     for name, t in (("q", q), ("k", k), ("v", v), ("q_dot", q_dot), ("k_dot", k_dot),
                     ("v_dot", v_dot)):
+        if t is None and name in ("k_dot", "v_dot"):
+            continue
         if not isinstance(t, torch.Tensor):
             raise TypeError(f"{name} must be a torch.Tensor")
         if t.dtype != torch.bfloat16:
@@ -93,7 +99,7 @@ def _check_inputs(q, k, v, q_dot, k_dot, v_dot):
     Lk = k.shape[2]
     for name, t, L in (("k", k, Lk), ("v", v, Lk), ("q_dot", q_dot, Lq), ("k_dot", k_dot, Lk),
                        ("v_dot", v_dot, Lk)):
-        if tuple(t.shape) != (B, H, L, d):
+        if t is not None and tuple(t.shape) != (B, H, L, d):
             raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {(B, H, L, d)}")
     return B, H, Lq, Lk, d
 
@@ -105,15 +111,18 @@ def _stream_handle(device, stream):
 
 
 def attn_jvp_fwd(q, k, v, q_dot, k_dot, v_dot, scale: float | None = None, kv_len=None,
-                 out=None, stream=None, *, _debug_timeout_ns: int | None = None,
-                 _debug_flags: int = 0):
+                 out=None, stream=None, *, lse_dot: bool = False,
+                 _debug_timeout_ns: int | None = None, _debug_flags: int = 0):
     """O = softmax(scale Q K^T) V, its tangent O' along (Q', K', V'), and lse.
 
     q, q_dot: bf16 [B, H, Lq, d]; k, v, k_dot, v_dot: bf16 [B, H, Lk, d];
     d in {64, 128}; kv_len: optional int32 [B] on the same device (keys
-    j >= kv_len[b] are masked).  scale defaults to 1/sqrt(d).  ``out`` may
-    supply (o, o_dot, lse) buffers.  Queued on ``stream`` (default: the
-    current stream).  Returns (o, o_dot, lse) with lse fp32 [B, H, Lq].
+    j >= kv_len[b] are masked).  scale defaults to 1/sqrt(d).  ``k_dot`` and
+    ``v_dot`` may both be None, meaning K' = V' = 0 (a cheaper kernel).  With
+    ``lse_dot=True`` the tangent of lse (sum_j P S') is returned as well.
+    ``out`` may supply (o, o_dot, lse[, lse_dot]) buffers.  Queued on
+    ``stream`` (default: the current stream).  Returns (o, o_dot, lse) or
+    (o, o_dot, lse, lse_dot), lse and lse_dot fp32 [B, H, Lq].
     """
     B, H, Lq, Lk, d = _check_inputs(q, k, v, q_dot, k_dot, v_dot)
     if scale is None:
@@ -125,24 +134,44 @@ def attn_jvp_fwd(q, k, v, q_dot, k_dot, v_dot, scale: float | None = None, kv_le
                 or not kv_len.is_contiguous()):
             raise ValueError("kv_len must be a contiguous int32 [B] tensor on q's device")
         kv_ptr = kv_len.data_ptr()
+    ld = None
     if out is None:
         o = torch.empty_like(q)
         od = torch.empty_like(q)
         lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+        if lse_dot:
+            ld = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
     else:
-        o, od, lse = out
+        if len(out) != (4 if lse_dot else 3):
+            raise ValueError("out must hold (o, o_dot, lse) or, with lse_dot, four buffers")
+        o, od, lse = out[:3]
+        if lse_dot:
+            ld = out[3]
+    for name, t in (("o", o), ("o_dot", od)):
+        if (t.dtype != torch.bfloat16 or t.device != q.device or not t.is_contiguous()
+                or tuple(t.shape) != (B, H, Lq, d)):
+            raise ValueError(f"{name} must be a contiguous bf16 [B, H, Lq, d] tensor on q's device")
+    for name, t in (("lse", lse), ("lse_dot", ld)):
+        if t is not None and (t.dtype != torch.float32 or t.device != q.device
+                              or not t.is_contiguous() or tuple(t.shape) != (B, H, Lq)):
+            raise ValueError(f"{name} must be a contiguous fp32 [B, H, Lq] tensor on q's device")
     lib = load_library()
-    ptrs = [t.data_ptr() for t in (q, k, v, q_dot, k_dot, v_dot, o, od, lse)]
+    ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    ptrs = [ptr(t) for t in (q, k, v, q_dot, k_dot, v_dot, o, od, lse)]
     sh = _stream_handle(q.device, stream)
     with torch.cuda.device(q.device):
-        if _debug_timeout_ns is None and not _debug_flags:
-            rc = lib.attn_jvp_fwd(*ptrs, B, H, Lq, Lk, d, float(scale), kv_ptr, sh)
-        else:
+        if _debug_timeout_ns is not None or _debug_flags:
+            if k_dot is None or lse_dot:
+                raise ValueError("the debug entry point takes all six inputs and no lse_dot")
             rc = lib.attn_jvp_fwd_debug(*ptrs, B, H, Lq, Lk, d, float(scale), kv_ptr, sh,
                                         int(_debug_timeout_ns or 0), int(_debug_flags))
+        elif k_dot is None or lse_dot:
+            rc = lib.attn_jvp_fwd_ex(*ptrs, ptr(ld), B, H, Lq, Lk, d, float(scale), kv_ptr, sh)
+        else:
+            rc = lib.attn_jvp_fwd(*ptrs, B, H, Lq, Lk, d, float(scale), kv_ptr, sh)
     if rc != ATTN_JVP_OK:
         raise AttnJvpError(rc, "attn_jvp_fwd")
-    return o, od, lse
+    return (o, od, lse, ld) if lse_dot else (o, od, lse)
 
 
 def attn_jvp_check(stream=None, device=None) -> tuple[int, int]:

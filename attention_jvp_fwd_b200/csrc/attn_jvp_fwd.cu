@@ -132,6 +132,7 @@ struct Params {
     void *o;
     void *od;
     float *lse;
+    float *lse_dot;  // NULL: not computed
     const int32_t *kv_len;
     int H, Lq, Lk, nqt;
     float scale;  // s
@@ -210,10 +211,14 @@ __device__ __forceinline__ float row_min64(const uint32_t (&a)[32], const uint32
     return row_ext64<true>(a, b);
 }
 
-template <int D, bool PAIR>
+// ZKV: K' = V' = 0 (frozen keys and values, e.g. text tokens).  Then S'_raw
+// = Q' K^T and O' = P' V: the K' and V' tiles are neither loaded nor
+// multiplied, 8 of the 12 FLOP units remain.
+template <int D, bool PAIR, bool ZKV>
 __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
     attn_jvp_fwd_kernel(const __grid_constant__ Params p)
 {
+    static_assert(!(PAIR && ZKV), "the CTA-pair layout always carries K' and V'");
     using C = Cfg<D, PAIR>;
     extern __shared__ __align__(1024) uint8_t smem[];
     // The 128-byte swizzle atoms must start on 1024-byte boundaries.  The
@@ -286,9 +291,11 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_qd);
         tma_prefetch_desc(&p.tm_k);
-        tma_prefetch_desc(&p.tm_kd);
         tma_prefetch_desc(&p.tm_v);
-        tma_prefetch_desc(&p.tm_vd);
+        if (!ZKV) {
+            tma_prefetch_desc(&p.tm_kd);
+            tma_prefetch_desc(&p.tm_vd);
+        }
         if (PAIR) tma_prefetch_desc(&p.tm_k32);
     }
     if (warp == 1) {
@@ -366,13 +373,14 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                                              j * BN + static_cast<int>(rank) * (BN / 2), bh, pol_kv);
                         }
                     } else {
-                        mbar_arrive_expect_tx(&k_full[s], C::KST_BYTES);
+                        mbar_arrive_expect_tx(&k_full[s], ZKV ? C::KST_BYTES / 2 : C::KST_BYTES);
 #pragma unroll
                         for (int c = 0; c < C::NKB; ++c) {
                             tma_load_3d(dst + c * (2 * BN * 128), &p.tm_k, &k_full[s], c * 64, j * BN, bh,
                                         pol_kv);
-                            tma_load_3d(dst + c * (2 * BN * 128) + BN * 128, &p.tm_kd, &k_full[s], c * 64,
-                                        j * BN, bh, pol_kv);
+                            if (!ZKV)
+                                tma_load_3d(dst + c * (2 * BN * 128) + BN * 128, &p.tm_kd, &k_full[s], c * 64,
+                                            j * BN, bh, pol_kv);
                         }
                     }
                     ++nk;
@@ -384,7 +392,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                         ok = wait_bar(&v_empty[s], ((jj / C::NV) - 1) & 1, wc, SITE_V_EMPTY, true, PAIR);
                     if (!ok) break;
                     uint8_t *dst = smem + C::OFF_V + s * C::VST_BYTES;
-                    mbar_arrive_expect_tx(&v_full[s], C::VST_BYTES);
+                    mbar_arrive_expect_tx(&v_full[s], ZKV ? C::VHALF_BYTES : C::VST_BYTES);
                     if constexpr (PAIR) {
                         // this CTA's 64-column half of V and V' (local barrier)
                         const int c0 = static_cast<int>(rank) * 64;
@@ -394,8 +402,9 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
 #pragma unroll
                         for (int c = 0; c < C::NKB; ++c) {
                             tma_load_3d(dst + c * (BN * 128), &p.tm_v, &v_full[s], c * 64, jj * BN, bh, pol_kv);
-                            tma_load_3d(dst + (C::NKB + c) * (BN * 128), &p.tm_vd, &v_full[s], c * 64, jj * BN,
-                                        bh, pol_kv);
+                            if (!ZKV)
+                                tma_load_3d(dst + (C::NKB + c) * (BN * 128), &p.tm_vd, &v_full[s], c * 64,
+                                            jj * BN, bh, pol_kv);
                         }
                     }
                     ++nv;
@@ -467,21 +476,22 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                     mma_commit_pair_mc(&k_empty[s], 0x3);
                     mma_commit_pair_mc(&s_full[j & 1], 0x3);
                 } else {
-                    // S | Q K'^T  =  Q [K ; K']^T   (N = 2 BN)
+                    // S | Q K'^T  =  Q [K ; K']^T   (N = 2 BN); with K' = 0 only
+                    // S = Q K^T (N = BN)
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
                         const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
                         mma_ss(tS, desc_add(dq, oa), desc_add(dk, ob),
-                               C::IDESC_S, kk > 0 ? 1u : 0u);
+                               ZKV ? C::IDESC_SD : C::IDESC_S, kk > 0 ? 1u : 0u);
                     }
-                    // += Q' K^T into the second half
+                    // += Q' K^T into the second half (with K' = 0 it starts it)
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t oa = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
                         const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
                         mma_ss(tS + BN, desc_add(dqd, oa), desc_add(dk, ob),
-                               C::IDESC_SD, 1u);
+                               C::IDESC_SD, (!ZKV || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(&k_empty[s]);
                     mma_commit(&s_full[j & 1]);
@@ -500,6 +510,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                 const uint32_t tP = tbase + C::T_S + (jj & 1) * (2 * BN);
                 const uint64_t dv = sdesc_sw128(smem_addr(smem + C::OFF_V + s * C::VST_BYTES), LBO, 1024);
                 const uint64_t dvd = desc_add(dv, C::VHALF_BYTES);
+                (void)dvd;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {  // O += P V
                     const uint32_t a = tP + C::t_pk(kk, false);
@@ -507,12 +518,14 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                     if constexpr (PAIR) mma_ts_pair(tbase + C::T_O, a, desc_add(dv, kk * 2048), C::IDESC_PV, acc);
                     else mma_ts(tbase + C::T_O, a, desc_add(dv, kk * 2048), C::IDESC_PV, acc);
                 }
+                if constexpr (!ZKV) {
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P V'
-                    const uint32_t a = tP + C::t_pk(kk, false);
-                    const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
-                    if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, desc_add(dvd, kk * 2048), C::IDESC_PV, acc);
-                    else mma_ts(tbase + C::T_OD, a, desc_add(dvd, kk * 2048), C::IDESC_PV, acc);
+                    for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P V'
+                        const uint32_t a = tP + C::t_pk(kk, false);
+                        const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+                        if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, desc_add(dvd, kk * 2048), C::IDESC_PV, acc);
+                        else mma_ts(tbase + C::T_OD, a, desc_add(dvd, kk * 2048), C::IDESC_PV, acc);
+                    }
                 }
             };
             auto issue_pb = [&](const int jj) {
@@ -523,8 +536,10 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P(sS' - c) V
                     const uint32_t a = tP + C::t_pk(kk, true);
-                    if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, desc_add(dv, kk * 2048), C::IDESC_PV, 1u);
-                    else mma_ts(tbase + C::T_OD, a, desc_add(dv, kk * 2048), C::IDESC_PV, 1u);
+                    // with V' = 0 this group starts O'_acc
+                    const uint32_t acc = (!ZKV || jj > 0 || kk > 0) ? 1u : 0u;
+                    if constexpr (PAIR) mma_ts_pair(tbase + C::T_OD, a, desc_add(dv, kk * 2048), C::IDESC_PV, acc);
+                    else mma_ts(tbase + C::T_OD, a, desc_add(dv, kk * 2048), C::IDESC_PV, acc);
                 }
                 if constexpr (PAIR) {
                     mma_commit_pair_mc(&v_empty[s], 0x3);
@@ -605,6 +620,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4 *>(out_ptr)[c] = z;
                 if (g == 0) p.lse[static_cast<size_t>(bh) * p.Lq + grow] = -INFINITY;
+                if (g == 1 && p.lse_dot) p.lse_dot[static_cast<size_t>(bh) * p.Lq + grow] = 0.f;
             }
         } else {
             const float sl2 = p.sl2;
@@ -745,7 +761,7 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                         tmem_st32(tacc + c, t);
                     }
                 }
-                if (!PAIR && tail) {
+                if (!PAIR && tail && !(ZKV && g == 1)) {  // (no V' tile with V' = 0)
                     // Zero the V (g = 0) / V' (g = 1) rows of padded keys so
                     // their bits (NaN included) cannot reach the PV products.
                     // Each warp zeroes its share and fences before it signals P.
@@ -858,6 +874,9 @@ __global__ void __launch_bounds__(Cfg<D, PAIR>::NTHREADS, 1)
                 }
                 if (g == 0 && grow < p.Lq)
                     p.lse[static_cast<size_t>(bh) * p.Lq + grow] = (m_used + log2f(lt)) * 0.69314718055994531f;
+                // lse' = sum_j P_j s S'_j = c + a / l
+                if (g == 1 && p.lse_dot && grow < p.Lq)
+                    p.lse_dot[static_cast<size_t>(bh) * p.Lq + grow] = cctr + coef;
             }
         }
     }
@@ -918,7 +937,7 @@ static bool make_map(CUtensorMap *m, const void *base, int D, int L, long long B
 
 constexpr int MAX_DEVICES = 64;
 
-template <int D, bool PAIR>
+template <int D, bool PAIR, bool ZKV>
 static int prepare_device(int dev)
 {
     static std::mutex mu;
@@ -926,7 +945,7 @@ static int prepare_device(int dev)
     if (dev < 0 || dev >= MAX_DEVICES) return ATTN_JVP_ERR_LAUNCH;
     std::lock_guard<std::mutex> g(mu);
     if (!done[dev]) {
-        if (cudaFuncSetAttribute(attn_jvp_fwd_kernel<D, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(attn_jvp_fwd_kernel<D, PAIR, ZKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(Cfg<D, PAIR>::SMEM_BYTES)) != cudaSuccess)
             return ATTN_JVP_ERR_LAUNCH;
         done[dev] = true;
@@ -934,12 +953,12 @@ static int prepare_device(int dev)
     return ATTN_JVP_OK;
 }
 
-template <int D, bool PAIR>
+template <int D, bool PAIR, bool ZKV>
 static int launch_kernel(const Params &prm, long long grid, cudaStream_t s)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
-    if (int rc = prepare_device<D, PAIR>(dev)) return rc;
+    if (int rc = prepare_device<D, PAIR, ZKV>(dev)) return rc;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -955,7 +974,7 @@ static int launch_kernel(const Params &prm, long long grid, cudaStream_t s)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    if (cudaLaunchKernelEx(&cfg, attn_jvp_fwd_kernel<D, PAIR>, prm) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
+    if (cudaLaunchKernelEx(&cfg, attn_jvp_fwd_kernel<D, PAIR, ZKV>, prm) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     return ATTN_JVP_OK;
 }
 
@@ -965,11 +984,15 @@ static bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb)
     return x < y + nb && y < x + na;
 }
 
+// allow_zero_kv: k_dot and v_dot may both be NULL (K' = V' = 0).
 static int launch(const void *q, const void *k, const void *v, const void *qd, const void *kd,
-                  const void *vd, void *o, void *od, float *lse, int B, int H, int Lq, int Lk, int d,
-                  float scale, const int32_t *kv_len, void *stream, uint64_t timeout_ns, int flags)
+                  const void *vd, void *o, void *od, float *lse, float *lse_dot, int B, int H, int Lq,
+                  int Lk, int d, float scale, const int32_t *kv_len, void *stream, uint64_t timeout_ns,
+                  int flags, bool allow_zero_kv)
 {
-    if (!q || !k || !v || !qd || !kd || !vd || !o || !od || !lse) return ATTN_JVP_ERR_NULL;
+    const bool zkv = allow_zero_kv && !kd && !vd;
+    if (!q || !k || !v || !qd || (!zkv && (!kd || !vd)) || !o || !od || !lse) return ATTN_JVP_ERR_NULL;
+    if (flags & ~(ATTN_JVP_DEBUG_STARVE_Q | ATTN_JVP_DEBUG_CTA_PAIR)) return ATTN_JVP_ERR_VALUE;
     if (B < 1 || H < 1 || Lq < 1 || Lk < 1) return ATTN_JVP_ERR_SHAPE;
     const long long BH = static_cast<long long>(B) * H;
     if (BH * Lq >= (1ll << 31) || BH * Lk >= (1ll << 31)) return ATTN_JVP_ERR_SHAPE;
@@ -977,40 +1000,43 @@ static int launch(const void *q, const void *k, const void *v, const void *qd, c
     const void *t16[8] = {q, k, v, qd, kd, vd, o, od};
     for (const void *t : t16)
         if (reinterpret_cast<uintptr_t>(t) & 15) return ATTN_JVP_ERR_ALIGN;
-    if ((reinterpret_cast<uintptr_t>(lse) & 3) || (reinterpret_cast<uintptr_t>(kv_len) & 3))
+    if ((reinterpret_cast<uintptr_t>(lse) & 3) || (reinterpret_cast<uintptr_t>(lse_dot) & 3) ||
+        (reinterpret_cast<uintptr_t>(kv_len) & 3))
         return ATTN_JVP_ERR_ALIGN;
     if (!std::isfinite(scale)) return ATTN_JVP_ERR_VALUE;
     const size_t nq = static_cast<size_t>(BH) * Lq * d * 2, nk = static_cast<size_t>(BH) * Lk * d * 2;
     const size_t nl = static_cast<size_t>(BH) * Lq * 4;
     const void *ins[6] = {q, k, v, qd, kd, vd};
     const size_t insz[6] = {nq, nk, nk, nq, nk, nk};
-    const void *outs[3] = {o, od, lse};
-    const size_t outsz[3] = {nq, nq, nl};
-    for (int i = 0; i < 3; ++i) {
+    const void *outs[4] = {o, od, lse, lse_dot};
+    const size_t outsz[4] = {nq, nq, nl, nl};
+    for (int i = 0; i < 4; ++i) {
+        if (!outs[i]) continue;
         for (int j = 0; j < 6; ++j)
-            if (ranges_overlap(outs[i], outsz[i], ins[j], insz[j])) return ATTN_JVP_ERR_VALUE;
-        for (int j = i + 1; j < 3; ++j)
-            if (ranges_overlap(outs[i], outsz[i], outs[j], outsz[j])) return ATTN_JVP_ERR_VALUE;
+            if (ins[j] && ranges_overlap(outs[i], outsz[i], ins[j], insz[j])) return ATTN_JVP_ERR_VALUE;
+        for (int j = i + 1; j < 4; ++j)
+            if (outs[j] && ranges_overlap(outs[i], outsz[i], outs[j], outsz[j])) return ATTN_JVP_ERR_VALUE;
     }
 
     const int nqt = (Lq + BM - 1) / BM;
     // One CTA per query tile by default.  The CTA-pair layout (d = 128 only,
     // selected by a test flag) halves the per-SM operand traffic but couples
     // the two CTAs' pipelines; on B200 it measures slightly slower today.
-    const bool pair = d == 128 && (flags & ATTN_JVP_DEBUG_CTA_PAIR);
+    const bool pair = d == 128 && !zkv && (flags & ATTN_JVP_DEBUG_CTA_PAIR);
     const long long grid = pair ? 2ll * ((nqt + 1) / 2) * BH : static_cast<long long>(nqt) * BH;
     if (grid > INT_MAX) return ATTN_JVP_ERR_SHAPE;
 
     Params prm;
     std::memset(&prm, 0, sizeof prm);
     if (!make_map(&prm.tm_q, q, d, Lq, BH, BM) || !make_map(&prm.tm_qd, qd, d, Lq, BH, BM) ||
-        !make_map(&prm.tm_k, k, d, Lk, BH, BN) || !make_map(&prm.tm_kd, kd, d, Lk, BH, BN) ||
-        !make_map(&prm.tm_v, v, d, Lk, BH, BN) || !make_map(&prm.tm_vd, vd, d, Lk, BH, BN) ||
-        !make_map(&prm.tm_k32, k, d, Lk, BH, BN / 2))
+        !make_map(&prm.tm_k, k, d, Lk, BH, BN) || !make_map(&prm.tm_v, v, d, Lk, BH, BN) ||
+        (!zkv && (!make_map(&prm.tm_kd, kd, d, Lk, BH, BN) || !make_map(&prm.tm_vd, vd, d, Lk, BH, BN))) ||
+        (pair && !make_map(&prm.tm_k32, k, d, Lk, BH, BN / 2)))
         return ATTN_JVP_ERR_LAUNCH;
     prm.o = o;
     prm.od = od;
     prm.lse = lse;
+    prm.lse_dot = lse_dot;
     prm.kv_len = kv_len;
     prm.H = H;
     prm.Lq = Lq;
@@ -1023,9 +1049,10 @@ static int launch(const void *q, const void *k, const void *v, const void *qd, c
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int rc;
-    if (d == 64) rc = launch_kernel<64, false>(prm, grid, s);
-    else if (pair) rc = launch_kernel<128, true>(prm, grid, s);
-    else rc = launch_kernel<128, false>(prm, grid, s);
+    if (zkv) rc = d == 64 ? launch_kernel<64, false, true>(prm, grid, s) : launch_kernel<128, false, true>(prm, grid, s);
+    else if (d == 64) rc = launch_kernel<64, false, false>(prm, grid, s);
+    else if (pair) rc = launch_kernel<128, true, false>(prm, grid, s);
+    else rc = launch_kernel<128, false, false>(prm, grid, s);
     if (rc) return rc;
     if (cudaGetLastError() != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     return ATTN_JVP_OK;
@@ -1039,8 +1066,16 @@ int attn_jvp_fwd(const void *q, const void *k, const void *v, const void *q_dot,
                  const void *v_dot, void *o, void *o_dot, float *lse, int B, int H, int Lq, int Lk,
                  int d, float scale, const int32_t *kv_len, void *stream)
 {
-    return ajvp::launch(q, k, v, q_dot, k_dot, v_dot, o, o_dot, lse, B, H, Lq, Lk, d, scale, kv_len,
-                        stream, 0, 0);
+    return ajvp::launch(q, k, v, q_dot, k_dot, v_dot, o, o_dot, lse, nullptr, B, H, Lq, Lk, d, scale,
+                        kv_len, stream, 0, 0, false);
+}
+
+int attn_jvp_fwd_ex(const void *q, const void *k, const void *v, const void *q_dot, const void *k_dot,
+                    const void *v_dot, void *o, void *o_dot, float *lse, float *lse_dot, int B, int H,
+                    int Lq, int Lk, int d, float scale, const int32_t *kv_len, void *stream)
+{
+    return ajvp::launch(q, k, v, q_dot, k_dot, v_dot, o, o_dot, lse, lse_dot, B, H, Lq, Lk, d, scale,
+                        kv_len, stream, 0, 0, true);
 }
 
 int attn_jvp_fwd_debug(const void *q, const void *k, const void *v, const void *q_dot,
@@ -1048,8 +1083,8 @@ int attn_jvp_fwd_debug(const void *q, const void *k, const void *v, const void *
                        int H, int Lq, int Lk, int d, float scale, const int32_t *kv_len, void *stream,
                        uint64_t timeout_ns, int flags)
 {
-    return ajvp::launch(q, k, v, q_dot, k_dot, v_dot, o, o_dot, lse, B, H, Lq, Lk, d, scale, kv_len,
-                        stream, timeout_ns, flags);
+    return ajvp::launch(q, k, v, q_dot, k_dot, v_dot, o, o_dot, lse, nullptr, B, H, Lq, Lk, d, scale,
+                        kv_len, stream, timeout_ns, flags, false);
 }
 
 int attn_jvp_check(void *stream, int *site)
@@ -1081,6 +1116,6 @@ const char *attn_jvp_status_string(int status)
     }
 }
 
-int attn_jvp_version(void) { return 100; }
+int attn_jvp_version(void) { return 200; }
 
 }  // extern "C"

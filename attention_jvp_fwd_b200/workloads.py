@@ -64,6 +64,11 @@ class Workload:
     def inputs(self):
         return self.q, self.k, self.v, self.q_dot, self.k_dot, self.v_dot
 
+    @property
+    def zero_kv_dot(self) -> bool:
+        """K' = V' = 0 for every batch (the zero-tangent kernel applies)."""
+        return bool(self.meta.get("zero_kv_dot", False))
+
     def flops_nominal(self) -> float:
         """12 * Lq * Lk * d per (b, h)."""
         return 12.0 * self.Lq * self.Lk * self.d * self.B * self.H
@@ -74,6 +79,11 @@ class Workload:
             return self.flops_nominal()
         n = np.clip(self.kv_len.astype(np.int64), 0, self.Lk)
         return float(12.0 * self.Lq * self.d * self.H * n.sum())
+
+    def flops_performed(self) -> float:
+        """FLOPs the kernel runs on the valid keys: 12 units, or 8 when
+        K' = V' = 0 lets it skip Q K'^T and P V'."""
+        return self.flops_valid() * (8.0 / 12.0 if self.zero_kv_dot else 1.0)
 
 
 def _normal(rng: np.random.Generator, shape, chunk: int = 1 << 24) -> np.ndarray:
@@ -151,6 +161,8 @@ def make_custom(B: int, H: int, Lq: int, Lk: int, d: int, seed: int = 0, *,
     if zero_kv_dot_from is not None:
         kd[zero_kv_dot_from:] = 0.0
         vd[zero_kv_dot_from:] = 0.0
+        # every batch frozen: callers may pass K' = V' = None
+        meta["zero_kv_dot"] = zero_kv_dot_from == 0
     if kv_len is not None:
         kv_len = np.asarray(kv_len, dtype=np.int32).reshape(B)
     return Workload(name, B, H, Lq, Lk, d, scale, _to_bits(q), _to_bits(k), _to_bits(v),
@@ -180,6 +192,8 @@ NAMED = {
     "t2i_self": dict(B=2, H=16, Lq=4096, Lk=4096, d=128),
     # T2I/T2V cross-attention to 512 text tokens with per-batch valid length
     "cross": dict(B=4, H=16, Lq=4096, Lk=512, d=128),
+    # the same with every batch's keys and values frozen (K' = V' = 0)
+    "cross_frozen": dict(B=4, H=16, Lq=4096, Lk=512, d=128),
     # T2V self-attention, 21 latent frames x 30 x 52 patches (14B-DiT-like)
     "t2v_self": dict(B=1, H=40, Lq=32760, Lk=32760, d=128),
 }
@@ -206,6 +220,7 @@ def make(name: str, seed: int = 0) -> Workload:
       tangents i.i.d. N(0, 1).
     - ``cross``: all N(0, 1); kv_len[b] ~ U{64..512}; K' = V' = 0 for the
       second half of the batch (frozen text tokens).
+    - ``cross_frozen``: as ``cross`` with K' = V' = 0 for every batch.
     - ``t2v_self``: Q, K rows at unit RMS; V and tangents N(0, 1).
     - ``stress_d{d}_L{L}``: Q x 4; tangents x 10**u, u ~ U[-3, 1] per head.
     - ``stress_sharp_d{d}_L{L}``: as stress but Q x 10, which puts the logit
@@ -218,11 +233,11 @@ def make(name: str, seed: int = 0) -> Workload:
     if name == "t2i_self":
         return make_custom(B, H, Lq, Lk, d, seed, name=name, unit_rms_qk=True,
                            head_gain_sd=0.1)
-    if name == "cross":
+    if name in ("cross", "cross_frozen"):
         rng = np.random.default_rng([seed, 7])
         kv = rng.integers(64, 513, size=B).astype(np.int32)
         return make_custom(B, H, Lq, Lk, d, seed, name=name, kv_len=kv,
-                           zero_kv_dot_from=B // 2)
+                           zero_kv_dot_from=B // 2 if name == "cross" else 0)
     if name == "t2v_self":
         return make_custom(B, H, Lq, Lk, d, seed, name=name, unit_rms_qk=True)
     if name.startswith("stress_sharp_"):

@@ -85,6 +85,34 @@ int attn_jvp_fwd(const void *q, const void *k, const void *v,
                  const int32_t *kv_len, void *stream);
 
 /*
+ * attn_jvp_fwd_ex -- attn_jvp_fwd with two additions.
+ *
+ *   lse_dot       fp32 device pointer [B, H, Lq], written, or NULL.  It
+ *                 receives the tangent of lse along (Q', K'):
+ *                 lse'_i = sum_j P_ij S'_ij (the row mean mu of the JVP
+ *                 above; d lse_i = sum_j P_ij dS_ij).  Rows with n_b = 0
+ *                 get 0.  It is formed as c + a / l from the kernel's running
+ *                 sums, so its error is of the order of the bf16 rounding of
+ *                 P (s S' - c) relative to the spread of s S' over the row.
+ *   k_dot, v_dot  may both be NULL, meaning K' = V' = 0 (keys and values that
+ *                 do not move, such as text tokens in cross-attention).
+ *                 Then S' = s Q' K^T and O' = P' V; the kernel neither loads
+ *                 nor multiplies K' and V', which removes 4 of the 12 FLOP
+ *                 units.  Exactly one of them NULL is ATTN_JVP_ERR_NULL.
+ *
+ * Everything else (layout, masking, ownership, errors) is as for
+ * attn_jvp_fwd; lse_dot must not overlap any other tensor.  The row mean
+ * and the zero-tangent case are the "next" items the rCM pages' kernel
+ * needs for cross-attention with frozen text keys (ai.info AI summary, Key
+ * Contributions 1: self- and cross-attention).
+ */
+int attn_jvp_fwd_ex(const void *q, const void *k, const void *v,
+                    const void *q_dot, const void *k_dot, const void *v_dot,
+                    void *o, void *o_dot, float *lse, float *lse_dot,
+                    int B, int H, int Lq, int Lk, int d, float scale,
+                    const int32_t *kv_len, void *stream);
+
+/*
  * attn_jvp_check -- synchronise `stream`, then read and clear the current
  * device's status word.  Returns ATTN_JVP_OK, ATTN_JVP_ERR_TIMEOUT if a
  * kernel launched since the last check gave up on a pipeline wait (its
@@ -102,7 +130,8 @@ const char *attn_jvp_status_string(int status);
  * and fault-injection flags, so a test can make a device-side wait run out
  * without hanging or faulting the GPU.
  *   timeout_ns  limit for every device-side wait (0 = the default, 2 s)
- *   flags       ATTN_JVP_DEBUG_* bits; 0 behaves exactly like attn_jvp_fwd
+ *   flags       ATTN_JVP_DEBUG_* bits; 0 behaves exactly like attn_jvp_fwd;
+ *               any other bit is ATTN_JVP_ERR_VALUE
  * No counterpart on the pages: it exists to test the failure path.
  */
 #define ATTN_JVP_DEBUG_STARVE_Q 1    /* never load Q/Q': the first wait on it runs out */
@@ -114,7 +143,7 @@ int attn_jvp_fwd_debug(const void *q, const void *k, const void *v,
                        const int32_t *kv_len, void *stream,
                        uint64_t timeout_ns, int flags);
 
-/* Library version, for logs: major*10000 + minor*100 + patch. */
+/* Library version, for logs: major*10000 + minor*100 + patch (0.2.0). */
 int attn_jvp_version(void);
 
 #ifdef __cplusplus

@@ -87,3 +87,47 @@ def test_python_binding_rejects_cpu_tensors():
         api.attn_jvp_fwd(q, q, q, q, q, q)
     with pytest.raises(TypeError):
         api.attn_jvp_fwd(q.float(), q, q, q, q, q)
+
+
+def _call_ex(lib, ptrs, lse_dot=None, B=1, H=1, Lq=1, Lk=1, d=64, scale=0.125):
+    return lib.attn_jvp_fwd_ex(*[ctypes.c_void_p(p) if p else None for p in ptrs],
+                               ctypes.c_void_p(lse_dot) if lse_dot else None, B, H, Lq, Lk, d,
+                               ctypes.c_float(scale), None, None)
+
+
+def test_ex_argument_errors(lib):
+    """attn_jvp_fwd_ex: k_dot and v_dot may be NULL together, not alone;
+    lse_dot is checked for alignment and overlap like the other outputs."""
+    good = [0x100000 * (i + 1) for i in range(9)]
+    for i in (4, 5):  # exactly one of k_dot, v_dot missing
+        bad = list(good)
+        bad[i] = 0
+        assert _call_ex(lib, bad) == api.ATTN_JVP_ERR_NULL
+    for i in (0, 1, 2, 3, 6, 7, 8):
+        bad = list(good)
+        bad[i] = 0
+        assert _call_ex(lib, bad) == api.ATTN_JVP_ERR_NULL
+    assert _call_ex(lib, good, lse_dot=0x2000002) == api.ATTN_JVP_ERR_ALIGN
+    assert _call_ex(lib, good, lse_dot=good[8]) == api.ATTN_JVP_ERR_VALUE  # lse_dot == lse
+    assert _call_ex(lib, good, lse_dot=good[0]) == api.ATTN_JVP_ERR_VALUE  # overlaps q
+    zero_kv = list(good)
+    zero_kv[4] = zero_kv[5] = 0
+    assert _call_ex(lib, zero_kv, d=96) == api.ATTN_JVP_ERR_HEADDIM  # reaches the later checks
+    # the plain entry point keeps requiring both tangents
+    assert _call(lib, zero_kv) == api.ATTN_JVP_ERR_NULL
+
+
+def test_debug_rejects_unknown_flags(lib):
+    good = [0x100000 * (i + 1) for i in range(9)]
+    rc = lib.attn_jvp_fwd_debug(*[ctypes.c_void_p(p) for p in good], 1, 1, 1, 1, 64,
+                                ctypes.c_float(0.125), None, None, ctypes.c_uint64(0), 1 << 5)
+    assert rc == api.ATTN_JVP_ERR_VALUE
+
+
+def test_python_binding_zero_tangent_arguments():
+    import torch
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):  # only one of k_dot, v_dot given
+        api.attn_jvp_fwd(q, q, q, q, q, None)
+    with pytest.raises(ValueError):  # CPU tensors, zero-tangent form
+        api.attn_jvp_fwd(q, q, q, q, None, None)
