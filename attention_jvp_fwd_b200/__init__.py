@@ -4,12 +4,13 @@
 (Q', K', V') and the row log-sum-exp, computed by hand-written sm_100a
 kernels behind a small C ABI (``include/attn_jvp.h``).  Importing this package
 does not load the CUDA library; the first call does, and fails loudly if it
-has not been built.
+has not been built.  ``scm_tangent_loss`` is the tangent-normalised sCM loss
+term that consumes such tangents.
 """
 from .api import (ATTN_JVP_ERR_ALIGN, ATTN_JVP_ERR_HEADDIM, ATTN_JVP_ERR_LAUNCH,  # noqa: F401
                   ATTN_JVP_ERR_NULL, ATTN_JVP_ERR_SHAPE, ATTN_JVP_ERR_TIMEOUT,
                   ATTN_JVP_ERR_VALUE, ATTN_JVP_OK, AttnJvpError, attn_jvp_check,
-                  attn_jvp_fwd, attn_jvp_status_string, library_path)
+                  attn_jvp_fwd, attn_jvp_status_string, library_path, scm_tangent_loss)
 
 __all__ = ["attn_jvp_fwd", "attn_jvp_check", "attn_jvp_status_string", "AttnJvpError",
-           "library_path"]
+           "library_path", "scm_tangent_loss"]

@@ -27,7 +27,7 @@ ATTN_JVP_DEBUG_STARVE_Q = 1
 ATTN_JVP_DEBUG_CTA_PAIR = 2
 
 EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_ex", "attn_jvp_fwd_debug", "attn_jvp_check",
-            "attn_jvp_status_string", "attn_jvp_version")
+            "attn_jvp_status_string", "attn_jvp_version", "scm_tangent_loss")
 
 _lock = threading.Lock()
 _lib = None
@@ -57,6 +57,8 @@ def load_library():
             vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
             lib.attn_jvp_fwd.restype = i32
             lib.attn_jvp_fwd.argtypes = [vp] * 9 + [i32] * 5 + [f32, vp, vp]
+            lib.scm_tangent_loss.restype = i32
+            lib.scm_tangent_loss.argtypes = [vp] * 5 + [i32, ctypes.c_longlong, f32, vp]
             lib.attn_jvp_fwd_ex.restype = i32
             lib.attn_jvp_fwd_ex.argtypes = [vp] * 10 + [i32] * 5 + [f32, vp, vp]
             lib.attn_jvp_fwd_debug.restype = i32
@@ -183,3 +185,45 @@ def attn_jvp_check(stream=None, device=None) -> tuple[int, int]:
     with torch.cuda.device(device):
         rc = lib.attn_jvp_check(_stream_handle(device, stream), ctypes.byref(site))
     return rc, site.value
+
+
+def scm_tangent_loss(f, f_ema, g, c: float = 0.1, grad: bool = True, out=None, stream=None):
+    """Tangent-normalised sCM loss per sample: r = F - F_ema - g / (|g|^2 + c),
+    loss = |r|^2 and (if ``grad``) d loss / dF = 2 r.
+
+    f, f_ema, g: contiguous bf16 CUDA tensors of one shape [B, ...] (each
+    sample flattened to N elements).  Returns ``(loss, grad)``: fp32 [B] and
+    bf16 of f's shape (None when ``grad`` is False).  ``out`` may supply
+    ``(loss, grad)`` buffers.
+    """
+    for name, t in (("f", f), ("f_ema", f_ema), ("g", g)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if t.shape != f.shape or t.device != f.device:
+            raise ValueError("f, f_ema and g must share one shape and device")
+    if f.dim() < 1 or f.numel() == 0:
+        raise ValueError("f must be [B, ...] with B >= 1 and at least one element per sample")
+    B = f.shape[0]
+    N = f.numel() // B
+    if out is None:
+        loss = torch.empty(B, dtype=torch.float32, device=f.device)
+        gr = torch.empty_like(f) if grad else None
+    else:
+        loss, gr = out
+    if loss.dtype != torch.float32 or tuple(loss.shape) != (B,) or loss.device != f.device:
+        raise ValueError("loss must be fp32 [B] on f's device")
+    if gr is not None and (gr.dtype != torch.bfloat16 or gr.shape != f.shape
+                           or not gr.is_contiguous() or gr.device != f.device):
+        raise ValueError("grad must be a contiguous bf16 tensor of f's shape")
+    lib = load_library()
+    with torch.cuda.device(f.device):
+        rc = lib.scm_tangent_loss(f.data_ptr(), f_ema.data_ptr(), g.data_ptr(), loss.data_ptr(),
+                                  None if gr is None else gr.data_ptr(), B, N, float(c),
+                                  _stream_handle(f.device, stream))
+    if rc != ATTN_JVP_OK:
+        raise AttnJvpError(rc, "scm_tangent_loss")
+    return loss, gr

@@ -130,6 +130,23 @@ __device__ __forceinline__ void cluster_sync()
                      "memory");
 }
 
+// Number of CTAs in this CTA's cluster.
+__device__ __forceinline__ uint32_t cluster_nctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// Load a float from shared memory given by its shared::cluster address
+// (this CTA's or a peer's, see mapa_shared).
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
 // Arrive once on an mbarrier given by its shared::cluster address (possibly
 // in the peer CTA), releasing this thread's prior writes at cluster scope.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)

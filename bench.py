@@ -443,8 +443,141 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------- sCM loss
+
+LOSS_METRIC = "sCM tangent-normalised loss GB/s (f, f_ema, g read once, grad written)"
+# T2V latents: Wan2.1 480p, 832x480x81 frames -> 16 channels x 21 x 60 x 104
+LOSS_SHAPE = (16, 16, 21, 60, 104)
+
+
+def loss_inputs(seed: int):
+    from attention_jvp_fwd_b200.workloads import bf16_round_bits
+    r = np.random.default_rng([seed, 11])
+    fe = r.standard_normal(LOSS_SHAPE, dtype=np.float32)
+    f = fe + np.float32(0.1) * r.standard_normal(LOSS_SHAPE, dtype=np.float32)
+    g = r.standard_normal(LOSS_SHAPE, dtype=np.float32)
+    return [bf16_round_bits(x) for x in (f, fe, g)]
+
+
+def run_loss(args):
+    """``--workload scm_loss``: the tangent-normalised sCM loss kernel, an
+    HBM-bound streaming reduction, on T2V-sized latents."""
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_setup()
+    group = ws > 1
+    if group:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from attention_jvp_fwd_b200.build import build
+    if rank == 0 or not group:
+        build()
+    if group:
+        dist.barrier()
+    import attention_jvp_fwd_b200 as A
+
+    bits = loss_inputs(args.seed + rank)
+    host = [torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).pin_memory() for b in bits]
+    ins = [h.to(dev, non_blocking=True) for h in host]
+    B = LOSS_SHAPE[0]
+    N = int(np.prod(LOSS_SHAPE[1:]))
+    loss = torch.empty(B, dtype=torch.float32, device=dev)
+    grad = torch.empty_like(ins[0])
+    stream = torch.cuda.Stream(dev)
+    bytes_step = 4.0 * B * N * 2 + 4 * B  # inputs > L2, so no flush is needed
+
+    def step():
+        A.scm_tangent_loss(*ins, out=(loss, grad), stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.6)
+    if group:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    local_ms = e0.elapsed_time(e1)
+    clocks = sampler.stop()
+    max_ms, total_bytes = aggregate(local_ms, bytes_step * args.steps, group, dev)
+    value = total_bytes / (max_ms * 1e-3) / 1e9
+
+    e2e_steps = args.e2e_steps or min(args.steps, 100)
+    hl = torch.empty(B, dtype=torch.float32, pin_memory=True)
+    hg = torch.empty(grad.shape, dtype=grad.dtype, pin_memory=True)
+    torch.cuda.synchronize(dev)
+    if group:
+        dist.barrier()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(e2e_steps):
+            for dst, src in zip(ins, host):
+                dst.copy_(src, non_blocking=True)
+            step()
+            hl.copy_(loss, non_blocking=True)
+            hg.copy_(grad, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms, e2e_bytes = aggregate(e0.elapsed_time(e1), bytes_step * e2e_steps, group, dev)
+
+    _, _, hbm, peak_src = load_peaks()
+    achieved = bytes_step / (local_ms / args.steps * 1e-3) / 1e9
+    line = {
+        "metric": LOSS_METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "scm_loss", "shape": list(LOSS_SHAPE), "c": 0.1, "seed": args.seed,
+                   "l2": "inputs exceed L2 (%.0f MB > 126 MB), no flush" % (3 * B * N * 2 / 1e6)
+                   if 3 * B * N * 2 > L2_BYTES else "inputs fit in L2: the number is L2-assisted"},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm,
+                     "peak_source": f"{peak_src} HBM copy bandwidth", "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "algorithmic_bytes": bytes_step,
+                     "kernel": "scm_loss_kernel<1>"},
+        "e2e": {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": 3 * B * N * 2, "d2h_bytes_per_step": B * N * 2 + 4 * B,
+                "steps": e2e_steps},
+        "clocks": clocks,
+    }
+    if rank == 0 and not group and not args.no_cpu_baseline:
+        from oracle import scm_loss
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < min(args.cpu_seconds, 10.0) or n == 0:
+            scm_loss.scm_tangent_loss(*[b[n % B:n % B + 1].reshape(1, -1) for b in bits])
+            n += 1
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n * 4.0 * N * 2 / dt / 1e9, "unit": "GB/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"{n} single-sample calls of numpy fp64, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if group:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.workload == "scm_loss":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the sCM loss leg has no reference arm; run the attention workloads"}))
+            return 0
+        return run_loss(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

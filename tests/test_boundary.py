@@ -11,6 +11,8 @@ from attention_jvp_fwd_b200.build import build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "attn_jvp.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if h.endswith(".h")]
 
 
 @pytest.fixture(scope="module")
@@ -20,9 +22,11 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(attn_jvp_\w+)\s*\(", text, re.M)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names.update(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*((?:attn_jvp|scm)_\w+)\s*\(", text, re.M))
+    return sorted(names)
 
 
 def test_header_declares_the_abi():
@@ -131,3 +135,33 @@ def test_python_binding_zero_tangent_arguments():
         api.attn_jvp_fwd(q, q, q, q, q, None)
     with pytest.raises(ValueError):  # CPU tensors, zero-tangent form
         api.attn_jvp_fwd(q, q, q, q, None, None)
+
+
+
+def test_scm_loss_argument_errors(lib):
+    good = [0x100000 * (i + 1) for i in range(5)]
+
+    def call(p, B=2, N=64, c=0.1):
+        return lib.scm_tangent_loss(*[ctypes.c_void_p(x) if x else None for x in p], B, N,
+                                    ctypes.c_float(c), None)
+    for i in range(4):
+        bad = list(good)
+        bad[i] = 0
+        assert call(bad) == api.ATTN_JVP_ERR_NULL
+    for B, N in [(0, 8), (2, 0), (70000, 8), (1, -1)]:
+        assert call(good, B, N) == api.ATTN_JVP_ERR_SHAPE
+    for i in (0, 1, 2, 4):
+        bad = list(good)
+        bad[i] += 8
+        assert call(bad) == api.ATTN_JVP_ERR_ALIGN
+    bad = list(good)
+    bad[3] += 2
+    assert call(bad) == api.ATTN_JVP_ERR_ALIGN
+    for c in (float("nan"), float("inf"), -0.5):
+        assert call(good, c=c) == api.ATTN_JVP_ERR_VALUE
+    alias = list(good)
+    alias[4] = alias[2]  # grad == g
+    assert call(alias) == api.ATTN_JVP_ERR_VALUE
+    alias = list(good)
+    alias[3] = alias[0] + 16  # loss inside f
+    assert call(alias) == api.ATTN_JVP_ERR_VALUE
