@@ -27,7 +27,8 @@ ATTN_JVP_DEBUG_STARVE_Q = 1
 ATTN_JVP_DEBUG_CTA_PAIR = 2
 
 EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_ex", "attn_jvp_fwd_debug", "attn_jvp_check",
-            "attn_jvp_status_string", "attn_jvp_version", "scm_tangent_loss")
+            "attn_jvp_status_string", "attn_jvp_version", "scm_tangent_loss", "qkv_rmsnorm_jvp",
+            "qkv_prologue_check")
 
 _lock = threading.Lock()
 _lib = None
@@ -57,6 +58,10 @@ def load_library():
             vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
             lib.attn_jvp_fwd.restype = i32
             lib.attn_jvp_fwd.argtypes = [vp] * 9 + [i32] * 5 + [f32, vp, vp]
+            lib.qkv_rmsnorm_jvp.restype = i32
+            lib.qkv_rmsnorm_jvp.argtypes = [vp] * 11 + [i32] * 5 + [f32, vp]
+            lib.qkv_prologue_check.restype = i32
+            lib.qkv_prologue_check.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
             lib.scm_tangent_loss.restype = i32
             lib.scm_tangent_loss.argtypes = [vp] * 5 + [i32, ctypes.c_longlong, f32, vp]
             lib.attn_jvp_fwd_ex.restype = i32
@@ -227,3 +232,51 @@ def scm_tangent_loss(f, f_ema, g, c: float = 0.1, grad: bool = True, out=None, s
     if rc != ATTN_JVP_OK:
         raise AttnJvpError(rc, "scm_tangent_loss")
     return loss, gr
+
+
+def qkv_rmsnorm_jvp(x, x_dot, w_qkv, gamma_q, gamma_k, B: int, L: int, H: int, eps: float = 1e-6,
+                    out=None, stream=None):
+    """QKV projection + per-head RMSNorm of tokens x and its tangent along x'.
+
+    x, x_dot: bf16 [B*L, D]; w_qkv: bf16 [3*H*d, D] (q, k, v heads stacked, as
+    a linear layer stores its weight); gamma_q, gamma_k: fp32 [d].  Returns
+    (q, k, v, q_dot, k_dot, v_dot), bf16 [B, H, L, d] each: the inputs of
+    attn_jvp_fwd.  ``out`` may supply the six buffers.
+    """
+    for name, t in (("x", x), ("x_dot", x_dot), ("w_qkv", w_qkv)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a bfloat16 torch.Tensor")
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 2:
+            raise ValueError(f"{name} must be a contiguous 2-D CUDA tensor")
+    for name, t in (("gamma_q", gamma_q), ("gamma_k", gamma_k)):
+        if (not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or not t.is_cuda
+                or not t.is_contiguous() or t.dim() != 1):
+            raise ValueError(f"{name} must be a contiguous fp32 1-D CUDA tensor")
+    T, D = x.shape
+    d = gamma_q.shape[0]
+    if T != B * L or x_dot.shape != x.shape or tuple(w_qkv.shape) != (3 * H * d, D) \
+            or gamma_k.shape != gamma_q.shape:
+        raise ValueError("shapes: x, x_dot [B*L, D], w_qkv [3*H*d, D], gamma_q, gamma_k [d]")
+    if out is None:
+        out = tuple(torch.empty((B, H, L, d), dtype=torch.bfloat16, device=x.device) for _ in range(6))
+    if len(out) != 6 or any(o.dtype != torch.bfloat16 or tuple(o.shape) != (B, H, L, d)
+                            or not o.is_contiguous() or o.device != x.device for o in out):
+        raise ValueError("out must be six contiguous bf16 [B, H, L, d] tensors on x's device")
+    lib = load_library()
+    with torch.cuda.device(x.device):
+        rc = lib.qkv_rmsnorm_jvp(x.data_ptr(), x_dot.data_ptr(), w_qkv.data_ptr(), gamma_q.data_ptr(),
+                                 gamma_k.data_ptr(), *[o.data_ptr() for o in out], B, L, H, D, d,
+                                 float(eps), _stream_handle(x.device, stream))
+    if rc != ATTN_JVP_OK:
+        raise AttnJvpError(rc, "qkv_rmsnorm_jvp")
+    return tuple(out)
+
+
+def qkv_prologue_check(stream=None, device=None) -> tuple[int, int]:
+    """Synchronise and read/clear the prologue kernel's status word: (status, site)."""
+    lib = load_library()
+    device = device if device is not None else torch.cuda.current_device()
+    site = ctypes.c_int(0)
+    with torch.cuda.device(device):
+        rc = lib.qkv_prologue_check(_stream_handle(device, stream), ctypes.byref(site))
+    return rc, site.value

@@ -12,9 +12,10 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = [os.path.join(CSRC, "attn_jvp_fwd.cu"), os.path.join(CSRC, "scm_loss.cu")]
+SOURCES = [os.path.join(CSRC, "attn_jvp_fwd.cu"), os.path.join(CSRC, "scm_loss.cu"),
+           os.path.join(CSRC, "qkv_prologue.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, "sm100.cuh"), os.path.join(ROOT, "include", "attn_jvp.h"),
-                  os.path.join(ROOT, "include", "scm_loss.h")]
+                  os.path.join(ROOT, "include", "scm_loss.h"), os.path.join(ROOT, "include", "qkv_prologue.h")]
 LIB_DIR = os.path.join(HERE, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libattn_jvp_fwd.so")
 

@@ -25,7 +25,7 @@ def declared_functions():
     names = set()
     for h in HEADERS:
         text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
-        names.update(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*((?:attn_jvp|scm)_\w+)\s*\(", text, re.M))
+        names.update(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*((?:attn_jvp|scm|qkv)_\w+)\s*\(", text, re.M))
     return sorted(names)
 
 
@@ -164,4 +164,37 @@ def test_scm_loss_argument_errors(lib):
     assert call(alias) == api.ATTN_JVP_ERR_VALUE
     alias = list(good)
     alias[3] = alias[0] + 16  # loss inside f
+    assert call(alias) == api.ATTN_JVP_ERR_VALUE
+
+
+
+def test_qkv_prologue_argument_errors(lib):
+    good = [0x100000 * (i + 1) for i in range(11)]
+
+    def call(p, B=1, L=128, H=2, D=256, d=128, eps=1e-6):
+        return lib.qkv_rmsnorm_jvp(*[ctypes.c_void_p(x) if x else None for x in p], B, L, H, D, d,
+                                   ctypes.c_float(eps), None)
+    for i in range(11):
+        bad = list(good)
+        bad[i] = 0
+        assert call(bad) == api.ATTN_JVP_ERR_NULL
+    for kw in ({"B": 0}, {"L": 0}, {"H": 0}, {"D": 0}, {"D": 96}, {"D": 32}):
+        assert call(good, **kw) == api.ATTN_JVP_ERR_SHAPE
+    for d in (32, 96, 256):
+        assert call(good, d=d) == api.ATTN_JVP_ERR_HEADDIM
+    for i in (0, 1, 2, 5, 6, 7, 8, 9, 10):
+        bad = list(good)
+        bad[i] += 8
+        assert call(bad) == api.ATTN_JVP_ERR_ALIGN
+    for i in (3, 4):
+        bad = list(good)
+        bad[i] += 2
+        assert call(bad) == api.ATTN_JVP_ERR_ALIGN
+    for eps in (float("nan"), -1.0):
+        assert call(good, eps=eps) == api.ATTN_JVP_ERR_VALUE
+    alias = list(good)
+    alias[5] = alias[0]  # q == x
+    assert call(alias) == api.ATTN_JVP_ERR_VALUE
+    alias = list(good)
+    alias[6] = alias[5] + 16  # q and k overlap
     assert call(alias) == api.ATTN_JVP_ERR_VALUE
