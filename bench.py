@@ -570,8 +570,131 @@ def run_loss(args):
     return 0
 
 
+# ----------------------------------------------------------------- QKV prologue
+
+QKV_METRIC = "QKV projection + RMSNorm forward-and-tangent TFLOP/s (2 GEMMs, 2*2*T*D*3*H*d)"
+# Cosmos-Predict2-2B-like layer on the T2I tokens: D = 2048, 16 heads of 128
+QKV_SHAPE = dict(B=2, L=4096, H=16, D=2048, d=128)
+
+
+def run_qkv(args):
+    """``--workload qkv_t2i``: the prologue kernel (a tensor-core GEMM pair with
+    an RMSNorm-JVP epilogue) on a T2I-sized layer."""
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_setup()
+    group = ws > 1
+    if group:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from attention_jvp_fwd_b200.build import build
+    if rank == 0 or not group:
+        build()
+    if group:
+        dist.barrier()
+    import attention_jvp_fwd_b200 as A
+    from attention_jvp_fwd_b200.workloads import bf16_round_bits
+
+    B, L, H, D, d = (QKV_SHAPE[k] for k in ("B", "L", "H", "D", "d"))
+    T = B * L
+    r = np.random.default_rng([args.seed + rank, 13])
+    bits = [bf16_round_bits(r.standard_normal((T, D), dtype=np.float32)),
+            bf16_round_bits(r.standard_normal((T, D), dtype=np.float32)),
+            bf16_round_bits((r.standard_normal((3 * H * d, D)) / np.sqrt(D)).astype(np.float32))]
+    host = [torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).pin_memory() for b in bits]
+    x, xd, w = (h.to(dev, non_blocking=True) for h in host)
+    gq = torch.ones(d, dtype=torch.float32, device=dev)
+    gk = torch.ones(d, dtype=torch.float32, device=dev)
+    outs = tuple(torch.empty((B, H, L, d), dtype=torch.bfloat16, device=dev) for _ in range(6))
+    stream = torch.cuda.Stream(dev)
+    flops_step = 2.0 * 2 * T * D * 3 * H * d
+
+    def step():
+        A.qkv_rmsnorm_jvp(x, xd, w, gq, gk, B, L, H, out=outs, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    st, site = A.qkv_prologue_check(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} at site {site}")
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.6)
+    if group:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    local_ms = e0.elapsed_time(e1)
+    clocks = sampler.stop()
+    max_ms, total = aggregate(local_ms, flops_step * args.steps, group, dev)
+    value = total / (max_ms * 1e-3) / 1e12
+
+    e2e_steps = args.e2e_steps or min(args.steps, 100)
+    hout = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(e2e_steps):
+            for dst, src in zip((x, xd, w), host):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for h, o in zip(hout, outs):
+                h.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms, e2e_fl = aggregate(e0.elapsed_time(e1), flops_step * e2e_steps, group, dev)
+
+    burst_tf, sustained_tf, _, peak_src = load_peaks()
+    if sustained_tf is not None and local_ms >= SUSTAINED_MS:
+        peak_tf, kind = sustained_tf, "sustained"
+    else:
+        peak_tf, kind = burst_tf, "burst"
+    achieved = flops_step / (local_ms / args.steps * 1e-3) / 1e12
+    in_bytes = sum(h.numel() * 2 for h in host)
+    line = {
+        "metric": QKV_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "qkv_t2i", **QKV_SHAPE, "seed": args.seed,
+                   "l2": "inputs %.0f MB; weights fit in L2 and are reused across token tiles, "
+                         "no flush" % (in_bytes / 1e6)},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf,
+                     "peak_source": f"{peak_src} bf16 dense ({kind}; timed region {local_ms:.0f} ms)",
+                     "unit": "TFLOP/s", "frac": achieved / peak_tf, "frac_of_burst_peak": achieved / burst_tf,
+                     "traffic": None, "flops_per_launch": flops_step,
+                     "kernel": "qkv_prologue_kernel<128>"},
+        "e2e": {"value": e2e_fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": sum(o.numel() * 2 for o in outs), "steps": e2e_steps},
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if group:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.workload == "qkv_t2i":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the prologue leg has no reference arm; run the attention workloads"}))
+            return 0
+        return run_qkv(args)
     if args.workload == "scm_loss":
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable":
