@@ -10,8 +10,9 @@
 //
 // The work is two streaming passes over HBM with one data-dependent scalar
 // between them, so the design is about bandwidth, not arithmetic:
-//   * one thread-block cluster per sample (16 CTAs where the GPU schedules
-//     them, else 8), each CTA a contiguous slice of the sample;
+//   * one thread-block cluster per sample, each CTA a contiguous slice of the
+//     sample; 8 or 16 CTAs per cluster, whichever finishes B samples in
+//     fewer cluster-waves per CTA (the GPU holds fewer 16-CTA clusters);
 //   * pass 1 sums g^2 in fp32; the CTAs meet at a cluster barrier and every
 //     CTA adds the slice sums from distributed shared memory in the same
 //     fixed order, so all hold the same n_b and the result is deterministic;
@@ -171,36 +172,61 @@ __global__ void __launch_bounds__(THREADS, 1)
     cluster_sync();  // no CTA leaves while CTA 0 may still read its shared memory
 }
 
+// How many clusters of `size` CTAs the GPU can hold at once (0 if none).
 template <bool VEC>
-static int cluster_size(int dev)
+static int max_active_clusters(int size)
+{
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(size), 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(size);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, scm_loss_kernel<VEC>, &cfg) != cudaSuccess) n = 0;
+    cudaGetLastError();  // a refused query leaves nothing behind
+    return n;
+}
+
+// Resident clusters of 8 and of 16 CTAs on this device (queried once).
+template <bool VEC>
+static void cluster_capacity(int dev, int &n8, int &n16)
 {
     static std::mutex mu;
-    static int cl[MAX_DEVICES] = {};
-    if (dev < 0 || dev >= MAX_DEVICES) return 0;
+    static int cap[MAX_DEVICES][2] = {};
+    static bool done[MAX_DEVICES] = {};
+    n8 = n16 = 0;
+    if (dev < 0 || dev >= MAX_DEVICES) return;
     std::lock_guard<std::mutex> lk(mu);
-    if (cl[dev] == 0) {
-        // 16 CTAs per cluster where the GPU can place them, else the portable 8
-        int size = 8;
+    if (!done[dev]) {
+        cap[dev][0] = max_active_clusters<VEC>(8);
         if (cudaFuncSetAttribute(scm_loss_kernel<VEC>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-            cudaSuccess) {
-            cudaLaunchConfig_t cfg;
-            std::memset(&cfg, 0, sizeof cfg);
-            cfg.gridDim = dim3(16, 1, 1);
-            cfg.blockDim = dim3(THREADS, 1, 1);
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = 16;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, scm_loss_kernel<VEC>, &cfg) == cudaSuccess && n > 0) size = 16;
-        }
-        cudaGetLastError();  // a refused probe leaves nothing behind
-        cl[dev] = size;
+            cudaSuccess)
+            cap[dev][1] = max_active_clusters<VEC>(16);
+        cudaGetLastError();
+        done[dev] = true;
     }
-    return cl[dev];
+    n8 = cap[dev][0];
+    n16 = cap[dev][1];
+}
+
+// Cluster size for B samples: each sample's time scales as 1 / size, and
+// the samples run in ceil(B / resident clusters) waves; take the smaller of
+// waves / size for 8 and 16 CTAs.
+template <bool VEC>
+static int cluster_size(int dev, int B)
+{
+    int n8, n16;
+    cluster_capacity<VEC>(dev, n8, n16);
+    if (n8 <= 0) return n16 > 0 ? 16 : 0;
+    if (n16 <= 0) return 8;
+    const long long w8 = (B + n8 - 1) / n8, w16 = (B + n16 - 1) / n16;
+    return (w16 * 8 < w8 * 16) ? 16 : 8;  // compare w16 / 16 with w8 / 8
 }
 
 static bool overlap(const void *a, size_t na, const void *b, size_t nb)
@@ -215,7 +241,7 @@ static int launch(const void *f, const void *fe, const void *g, float *loss, voi
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
-    const int cl = cluster_size<VEC>(dev);
+    const int cl = cluster_size<VEC>(dev, B);
     if (cl == 0) return ATTN_JVP_ERR_LAUNCH;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);

@@ -38,8 +38,12 @@ METRIC = ("attention fwd+JVP TFLOP/s (12·Lq·Lk·d/head) and % of B200 BF16 "
 UNIT = "TFLOP/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
+# the sources each timed kernel is built from (a traffic record counts only
+# while their hash is unchanged)
 KERNEL_SOURCES = ["attention_jvp_fwd_b200/csrc/attn_jvp_fwd.cu",
                   "attention_jvp_fwd_b200/csrc/sm100.cuh"]
+LOSS_SOURCES = ["attention_jvp_fwd_b200/csrc/scm_loss.cu", "attention_jvp_fwd_b200/csrc/sm100.cuh"]
+QKV_SOURCES = ["attention_jvp_fwd_b200/csrc/qkv_prologue.cu", "attention_jvp_fwd_b200/csrc/sm100.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -60,9 +64,9 @@ def parse_args(argv=None):
 
 # ----------------------------------------------------------------- helpers
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in sources or KERNEL_SOURCES:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -86,7 +90,7 @@ def load_peaks():
 SUSTAINED_MS = 500.0
 
 
-def measured_traffic(workload: str):
+def measured_traffic(workload: str, sources=None):
     """DRAM bytes per launch from a committed ncu capture, if it was taken on
     the current kernel source (else None)."""
     try:
@@ -95,7 +99,7 @@ def measured_traffic(workload: str):
     except (OSError, ValueError):
         return None
     e = t.get(workload)
-    if not e or e.get("source_sha256") != kernel_source_hash():
+    if not e or e.get("source_sha256") != kernel_source_hash(sources):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -544,7 +548,8 @@ def run_loss(args):
         "gpu_launches": args.steps,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm,
                      "peak_source": f"{peak_src} HBM copy bandwidth", "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "algorithmic_bytes": bytes_step,
+                     "frac": achieved / hbm, "traffic": measured_traffic("scm_loss", LOSS_SOURCES),
+                     "algorithmic_bytes": bytes_step,
                      "kernel": "scm_loss_kernel<1>"},
         "e2e": {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": 3 * B * N * 2, "d2h_bytes_per_step": B * N * 2 + 4 * B,
@@ -673,7 +678,7 @@ def run_qkv(args):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf,
                      "peak_source": f"{peak_src} bf16 dense ({kind}; timed region {local_ms:.0f} ms)",
                      "unit": "TFLOP/s", "frac": achieved / peak_tf, "frac_of_burst_peak": achieved / burst_tf,
-                     "traffic": None, "flops_per_launch": flops_step,
+                     "traffic": measured_traffic("qkv_t2i", QKV_SOURCES), "flops_per_launch": flops_step,
                      "kernel": "qkv_prologue_kernel<128>"},
         "e2e": {"value": e2e_fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": sum(o.numel() * 2 for o in outs), "steps": e2e_steps},
