@@ -15,13 +15,16 @@
 // and writes q, k, v, q', k', v' in the attention layout [B, H, L, d], so
 // the attention kernel reads them directly.
 //
-// One CTA computes a 128-token x one-head tile: two tcgen05 GEMMs that share
-// the weight tile, Y = X W_h^T and Y' = X' W_h^T (M = 128, N = d, K = D), with
-// both accumulators in TMEM.  A TMA warp streams X, X' and W_h in 64-column
-// slices through a 4-stage ring; one warp issues the MMAs; four epilogue
-// warps (thread = token) reduce each row's y^2 and y y' over the head, apply
-// the RMSNorm and its tangent, and store bf16.  Waits are bounded like the
-// attention kernel's (status word read by qkv_prologue_check).
+// A tile is 128 tokens x one head: two tcgen05 GEMMs that share the weight
+// tile, Y = X W_h^T and Y' = X' W_h^T (M = 128, N = d, K = D), both
+// accumulating in TMEM.  The kernel is persistent (one CTA per SM walks the
+// tiles) with two accumulator sets, so the epilogue of one tile overlaps the
+// MMAs of the next.  A TMA warp streams X, X' and W_h in 64-column slices
+// through a 4-stage ring that runs on across tiles; one warp issues the
+// MMAs; four epilogue warps (thread = token) reduce each row's y^2 and y y'
+// over the head, apply the RMSNorm and its tangent, and store bf16.  Waits
+// are bounded like the attention kernel's (status word read by
+// qkv_prologue_check).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -53,10 +56,10 @@ struct PCfg {
     static constexpr uint32_t B_BYTES = DH * BK * 2;   // W_h slice per stage
     static constexpr uint32_t ST_BYTES = 2 * A_BYTES + B_BYTES;
     static constexpr uint32_t OFF_BAR = NS * ST_BYTES;
-    static constexpr uint32_t OFF_MISC = OFF_BAR + (2 * NS + 1) * 8;  // tmem slot, abort
-    static constexpr uint32_t OFF_GAMMA = OFF_MISC + 16;              // float [DH]
-    static constexpr uint32_t SMEM_BYTES = OFF_GAMMA + DH * 4;
-    static constexpr uint32_t TMEM_COLS = 2 * DH;                      // Y | Y'
+    static constexpr uint32_t OFF_MISC = OFF_BAR + (2 * NS + 5) * 8;  // tmem slot, abort
+    static constexpr uint32_t OFF_GAMMA = OFF_MISC + 16;              // float [2][DH]
+    static constexpr uint32_t SMEM_BYTES = OFF_GAMMA + 2 * DH * 4;
+    static constexpr uint32_t TMEM_COLS = 4 * DH;                      // two sets of Y | Y'
     static constexpr uint32_t IDESC = idesc_bf16_f32(BM, DH, false);
     static_assert(SMEM_BYTES + 1024 <= 232448, "shared memory budget");
 };
@@ -65,7 +68,7 @@ struct Params {
     CUtensorMap tm_x, tm_xd, tm_w;
     const float *gamma_q, *gamma_k;
     __nv_bfloat16 *out[6];  // q, k, v, q', k', v'
-    int T, L, H, D;
+    int T, L, H, D, tiles_m;
     float eps;
     uint64_t timeout_ns;
 };
@@ -102,24 +105,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tiles_n = 3 * p.H;
-    const int nt = blockIdx.x % tiles_n;  // output channel block: part * H + head
-    const int mt = blockIdx.x / tiles_n;  // token tile
-    const int part = nt / p.H, head = nt % p.H;
+    const int n_tiles = p.tiles_m * tiles_n;
     const int nk = p.D / BK;
+    // this CTA's tiles: blockIdx.x, + gridDim.x, ...  (head tile fastest, so
+    // CTAs running together share the token tile through L2)
+    const int my_tiles = blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *empty = full + NS;
-    uint64_t *acc_full = empty + NS;
+    uint64_t *acc_full = empty + NS;  // [2] accumulator set b holds a finished tile
+    uint64_t *acc_empty = acc_full + 2;  // [2] the epilogue has read accumulator set b
+    uint64_t *drain = acc_empty + 2;     // MMAs in flight after an abort are done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
-    float *gamma = reinterpret_cast<float *>(smem + C::OFF_GAMMA);
+    float *gamma = reinterpret_cast<float *>(smem + C::OFF_GAMMA);  // [2][DH]: q, k
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+        }
+        mbar_init(drain, 1);
         *abort = 0;
         fence_barrier_init();
     }
@@ -127,9 +137,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp >= 2 && part < 2) {
-        const float *gsrc = part == 0 ? p.gamma_q : p.gamma_k;
-        for (int i = tid - 64; i < DH; i += 128) gamma[i] = gsrc[i];
+    if (warp >= 2) {
+        for (int i = tid - 64; i < 2 * DH; i += 128) gamma[i] = i < DH ? p.gamma_q[i] : p.gamma_k[i - DH];
     }
     tc_fence_before();
     __syncthreads();
@@ -137,53 +146,76 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
     const uint32_t tbase = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------------------------------------------------------- TMA
+        // ---------------------------------------------------------------- TMA: one ring across all tiles
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_last();
-            int issued = 0;
-            for (int k = 0; k < nk; ++k) {
-                const int s = k % NS;
-                if (k >= NS && !wait(&empty[s], ((k / NS) - 1) & 1, abort, p.timeout_ns, 1)) break;
-                uint8_t *st = smem + s * C::ST_BYTES;
-                mbar_arrive_expect_tx(&full[s], C::ST_BYTES);
-                tma_load_3d(st, &p.tm_x, &full[s], k * BK, mt * BM, 0, pol);
-                tma_load_3d(st + C::A_BYTES, &p.tm_xd, &full[s], k * BK, mt * BM, 0, pol);
-                tma_load_3d(st + 2 * C::A_BYTES, &p.tm_w, &full[s], k * BK, nt * DH, 0, pol);
-                issued = k + 1;
+            long long issued = 0;  // slices loaded so far
+            bool ok = true;
+            for (int li = 0; li < my_tiles && ok; ++li) {
+                const int t = blockIdx.x + li * gridDim.x;
+                const int nt = t % tiles_n, mt = t / tiles_n;
+                for (int k = 0; k < nk; ++k) {
+                    const int s = static_cast<int>(issued % NS);
+                    if (issued >= NS &&
+                        !wait(&empty[s], static_cast<uint32_t>((issued / NS) - 1) & 1, abort, p.timeout_ns, 1)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = smem + s * C::ST_BYTES;
+                    mbar_arrive_expect_tx(&full[s], C::ST_BYTES);
+                    tma_load_3d(st, &p.tm_x, &full[s], k * BK, mt * BM, 0, pol);
+                    tma_load_3d(st + C::A_BYTES, &p.tm_xd, &full[s], k * BK, mt * BM, 0, pol);
+                    tma_load_3d(st + 2 * C::A_BYTES, &p.tm_w, &full[s], k * BK, nt * DH, 0, pol);
+                    ++issued;
+                }
             }
             // let every load issued land before the CTA can exit (the last
             // phase of each stage, so the parity test is unambiguous)
-            for (int k = (issued > NS ? issued - NS : 0); k < issued; ++k)
-                wait(&full[k % NS], (k / NS) & 1, abort, p.timeout_ns, 2, false);
+            for (long long q = (issued > NS ? issued - NS : 0); q < issued; ++q)
+                wait(&full[q % NS], static_cast<uint32_t>(q / NS) & 1, abort, p.timeout_ns, 2, false);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA (warp-wide, elected lane)
         bool ok = true, issued = false;
-        for (int k = 0; k < nk && ok; ++k) {
-            const int s = k % NS;
-            ok = __all_sync(0xffffffffu, wait(&full[s], (k / NS) & 1, abort, p.timeout_ns, 3));
+        long long used = 0;  // slices consumed so far
+        for (int li = 0; li < my_tiles && ok; ++li) {
+            const int b = li & 1;
+            const uint32_t acc = tbase + b * (2 * DH);
+            if (li >= 2) {
+                ok = __all_sync(0xffffffffu, wait(&acc_empty[b], ((li >> 1) - 1) & 1, abort, p.timeout_ns, 6));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            for (int k = 0; k < nk; ++k, ++used) {
+                const int s = static_cast<int>(used % NS);
+                ok = __all_sync(0xffffffffu, wait(&full[s], static_cast<uint32_t>(used / NS) & 1, abort,
+                                                  p.timeout_ns, 3));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t st = smem_addr(smem + s * C::ST_BYTES);
+                const uint64_t dx = sdesc_sw128(st, 16, 1024);
+                const uint64_t dxd = sdesc_sw128(st + C::A_BYTES, 16, 1024);
+                const uint64_t dw = sdesc_sw128(st + 2 * C::A_BYTES, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    mma_ss(acc, desc_add(dx, kk * 32), desc_add(dw, kk * 32), C::IDESC,
+                           (k > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    mma_ss(acc + DH, desc_add(dxd, kk * 32), desc_add(dw, kk * 32), C::IDESC,
+                           (k > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&empty[s]);
+                issued = true;
+            }
             if (!ok) break;
-            tc_fence_after();
-            const uint32_t st = smem_addr(smem + s * C::ST_BYTES);
-            const uint64_t dx = sdesc_sw128(st, 16, 1024);
-            const uint64_t dxd = sdesc_sw128(st + C::A_BYTES, 16, 1024);
-            const uint64_t dw = sdesc_sw128(st + 2 * C::A_BYTES, 16, 1024);
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-                mma_ss(tbase, desc_add(dx, kk * 32), desc_add(dw, kk * 32), C::IDESC, (k > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-                mma_ss(tbase + DH, desc_add(dxd, kk * 32), desc_add(dw, kk * 32), C::IDESC,
-                       (k > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&empty[s]);
-            issued = true;
+            mma_commit(&acc_full[b]);
         }
-        if (issued) {
-            mma_commit(acc_full);
-            // after an abort nobody else waits for the MMAs in flight: do it
-            // here, so TMEM is not freed under them
-            if (!ok) wait(acc_full, 0, abort, p.timeout_ns, 5, false);
+        if (!ok && issued) {
+            // nobody else waits for the MMAs in flight after an abort: drain
+            // them here, so TMEM is not freed under them
+            mma_commit(drain);
+            wait(drain, 0, abort, p.timeout_ns, 5, false);
         }
         __syncwarp();
     } else {
@@ -191,72 +223,83 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-        const uint32_t ty = tbase + lane_off, tyd = tbase + lane_off + DH;
-        bool ok = wait(acc_full, 0, abort, p.timeout_ns, 4);
-        ok = __all_sync(0xffffffffu, ok && !*abort);  // warp-uniform: tcgen05.ld below is collective
-        tc_fence_after();
-        const int t = mt * BM + r;
-        if (ok) {
+        for (int li = 0; li < my_tiles; ++li) {
+            const int b = li & 1;
+            const int t_idx = blockIdx.x + li * gridDim.x;
+            const int nt = t_idx % tiles_n, mt = t_idx / tiles_n;
+            const int part = nt / p.H, head = nt % p.H;
+            const uint32_t ty = tbase + lane_off + b * (2 * DH), tyd = ty + DH;
+            bool ok = wait(&acc_full[b], (li >> 1) & 1, abort, p.timeout_ns, 4);
+            ok = __all_sync(0xffffffffu, ok && !*abort);  // warp-uniform: tcgen05.ld below is collective
+            if (!ok) break;
+            tc_fence_after();
+            const int t = mt * BM + r;
+            const float *g = gamma + (part == 1 ? DH : 0);
             float rs = 1.f, mix = 0.f;
             if (part < 2) {
                 // sums over the head's channels: y^2 and y y'
                 float s2 = 0.f, sm = 0.f;
 #pragma unroll 1
                 for (int c = 0; c < DH; c += 32) {
-                    uint32_t a[32], b[32];
+                    uint32_t a[32], e[32];
                     tmem_ld32(ty + c, a);
-                    tmem_ld32(tyd + c, b);
-                    tmem_ld_wait2(a, b);
+                    tmem_ld32(tyd + c, e);
+                    tmem_ld_wait2(a, e);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const float y = __uint_as_float(a[i]);
                         s2 = fmaf(y, y, s2);
-                        sm = fmaf(y, __uint_as_float(b[i]), sm);
+                        sm = fmaf(y, __uint_as_float(e[i]), sm);
                     }
                 }
                 rs = 1.f / sqrtf(s2 / DH + p.eps);
                 mix = rs * rs * rs * (sm / DH);  // r^3 mean(y y')
             }
-            // tcgen05.ld is warp-collective: every lane loads, only rows of real
-            // tokens store
-            {
-                const bool store = t < p.T;
-                const int tt = store ? t : 0;
-                const int bb = tt / p.L, l = tt % p.L;
-                const size_t o = ((static_cast<size_t>(bb) * p.H + head) * p.L + l) * DH;
-                __nv_bfloat16 *dy = p.out[part] + o;
-                __nv_bfloat16 *dyd = p.out[3 + part] + o;
+            // every lane loads (tcgen05.ld is warp-collective); only rows of
+            // real tokens store
+            const bool store = t < p.T;
+            const int tt = store ? t : 0;
+            const int bb = tt / p.L, l = tt % p.L;
+            const size_t o = ((static_cast<size_t>(bb) * p.H + head) * p.L + l) * DH;
+            __nv_bfloat16 *dy = p.out[part] + o;
+            __nv_bfloat16 *dyd = p.out[3 + part] + o;
 #pragma unroll 1
-                for (int c = 0; c < DH; c += 32) {
-                    uint32_t a[32], b[32], py[16], pyd[16];
-                    tmem_ld32(ty + c, a);
-                    tmem_ld32(tyd + c, b);
-                    tmem_ld_wait2(a, b);
+            for (int c = 0; c < DH; c += 32) {
+                uint32_t a[32], e[32], py[16], pyd[16];
+                tmem_ld32(ty + c, a);
+                tmem_ld32(tyd + c, e);
+                tmem_ld_wait2(a, e);
+                if (c + 32 == DH) {
+                    // the last read of this accumulator set: hand it back to
+                    // the MMA warp before the stores
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_empty[b]);
+                }
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float y0 = __uint_as_float(a[2 * i]), y1 = __uint_as_float(a[2 * i + 1]);
-                        float e0 = __uint_as_float(b[2 * i]), e1 = __uint_as_float(b[2 * i + 1]);
-                        if (part < 2) {
-                            const float g0 = gamma[c + 2 * i], g1 = gamma[c + 2 * i + 1];
-                            const float n0 = g0 * (e0 * rs - y0 * mix), n1 = g1 * (e1 * rs - y1 * mix);
-                            y0 = g0 * (y0 * rs);
-                            y1 = g1 * (y1 * rs);
-                            e0 = n0;
-                            e1 = n1;
-                        }
-                        uint32_t u, w;
-                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(y1), "f"(y0));
-                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(e1), "f"(e0));
-                        py[i] = u;
-                        pyd[i] = w;
+                for (int i = 0; i < 16; ++i) {
+                    float y0 = __uint_as_float(a[2 * i]), y1 = __uint_as_float(a[2 * i + 1]);
+                    float e0 = __uint_as_float(e[2 * i]), e1 = __uint_as_float(e[2 * i + 1]);
+                    if (part < 2) {
+                        const float g0 = g[c + 2 * i], g1 = g[c + 2 * i + 1];
+                        const float n0 = g0 * (e0 * rs - y0 * mix), n1 = g1 * (e1 * rs - y1 * mix);
+                        y0 = g0 * (y0 * rs);
+                        y1 = g1 * (y1 * rs);
+                        e0 = n0;
+                        e1 = n1;
                     }
-                    if (store) {
-                        uint4 *d0 = reinterpret_cast<uint4 *>(dy + c), *d1 = reinterpret_cast<uint4 *>(dyd + c);
+                    uint32_t u, w;
+                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(y1), "f"(y0));
+                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(e1), "f"(e0));
+                    py[i] = u;
+                    pyd[i] = w;
+                }
+                if (store) {
+                    uint4 *d0 = reinterpret_cast<uint4 *>(dy + c), *d1 = reinterpret_cast<uint4 *>(dyd + c);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            d0[i] = make_uint4(py[4 * i], py[4 * i + 1], py[4 * i + 2], py[4 * i + 3]);
-                            d1[i] = make_uint4(pyd[4 * i], pyd[4 * i + 1], pyd[4 * i + 2], pyd[4 * i + 3]);
-                        }
+                    for (int i = 0; i < 4; ++i) {
+                        d0[i] = make_uint4(py[4 * i], py[4 * i + 1], py[4 * i + 2], py[4 * i + 3]);
+                        d1[i] = make_uint4(pyd[4 * i], pyd[4 * i + 1], pyd[4 * i + 2], pyd[4 * i + 3]);
                     }
                 }
             }
@@ -350,8 +393,8 @@ int qkv_rmsnorm_jvp(const void *x, const void *x_dot, const void *w_qkv, const f
     if (d != 64 && d != 128) return ATTN_JVP_ERR_HEADDIM;
     const long long T = static_cast<long long>(B) * L;
     if (T >= (1ll << 31) || 3ll * H * d >= (1ll << 31)) return ATTN_JVP_ERR_SHAPE;
-    const long long grid = ((T + BM - 1) / BM) * 3ll * H;
-    if (grid > INT_MAX) return ATTN_JVP_ERR_SHAPE;
+    const long long n_tiles = ((T + BM - 1) / BM) * 3ll * H;
+    if (n_tiles > INT_MAX) return ATTN_JVP_ERR_SHAPE;
     const void *a16[9] = {x, x_dot, w_qkv, q, k, v, q_dot, k_dot, v_dot};
     for (const void *p : a16)
         if (reinterpret_cast<uintptr_t>(p) & 15) return ATTN_JVP_ERR_ALIGN;
@@ -381,9 +424,16 @@ int qkv_rmsnorm_jvp(const void *x, const void *x_dot, const void *w_qkv, const f
     prm.L = L;
     prm.H = H;
     prm.D = D;
+    prm.tiles_m = static_cast<int>((T + BM - 1) / BM);
     prm.eps = eps;
     prm.timeout_ns = TIMEOUT_NS;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // persistent: one CTA per SM (or per tile, if there are fewer)
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return ATTN_JVP_ERR_LAUNCH;
+    const long long grid = n_tiles < sms ? n_tiles : sms;
     return d == 128 ? launch_kernel<128>(prm, grid, s) : launch_kernel<64>(prm, grid, s);
 }
 
