@@ -24,7 +24,6 @@ ATTN_JVP_ERR_LAUNCH = -5
 ATTN_JVP_ERR_TIMEOUT = -6
 ATTN_JVP_ERR_VALUE = -7
 ATTN_JVP_DEBUG_STARVE_Q = 1
-ATTN_JVP_DEBUG_CTA_PAIR = 2
 
 EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_ex", "attn_jvp_fwd_debug", "attn_jvp_check",
             "attn_jvp_status_string", "attn_jvp_version", "scm_tangent_loss", "qkv_rmsnorm_jvp",

@@ -135,7 +135,6 @@ const char *attn_jvp_status_string(int status);
  * No counterpart on the pages: it exists to test the failure path.
  */
 #define ATTN_JVP_DEBUG_STARVE_Q 1    /* never load Q/Q': the first wait on it runs out */
-#define ATTN_JVP_DEBUG_CTA_PAIR 2    /* d = 128: CTA pairs (M = 256 MMAs) instead of one CTA per query tile */
 int attn_jvp_fwd_debug(const void *q, const void *k, const void *v,
                        const void *q_dot, const void *k_dot, const void *v_dot,
                        void *o, void *o_dot, float *lse,

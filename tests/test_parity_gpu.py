@@ -93,16 +93,18 @@ def test_named_workload_rows(name):
     print(name, m)
 
 
-@pytest.mark.parametrize("Lq,Lk,kv", [(300, 1000, None), (4096, 512, [512, 64, 300, 1]),
-                                       (129, 4099, None), (1, 64, [0])])
-def test_cta_pair_path(Lq, Lk, kv):
-    """d = 128 can also run as CTA pairs (M = 256 MMAs split over two SMs)."""
-    from attention_jvp_fwd_b200 import api
-    B = 1 if kv is None else len(kv)
-    w = W.make_custom(B, 2, Lq, Lk, 128, seed=12, kv_len=kv)
-    ins = [to_dev(x) for x in w.inputs()]
-    kvt = torch.from_numpy(w.kv_len).cuda() if w.kv_len is not None else None
-    o, od, lse = api.attn_jvp_fwd(*ins, scale=w.scale, kv_len=kvt,
-                                  _debug_flags=api.ATTN_JVP_DEBUG_CTA_PAIR)
-    torch.cuda.synchronize()
-    compare(gpu_rows(o, od, lse), oracle_ref(w), f"CTA pair Lq{Lq} Lk{Lk}")
+@pytest.mark.parametrize("d", [64, 128])
+def test_persistent_tile_walk(d):
+    """More query tiles (288) than SMs, so every CTA walks several of them and
+    the K/V rings, the S buffers and the barrier phases carry on from one
+    query tile to the next; batches without keys (which every role skips)
+    sit between ones with full, tail and single-key lengths, and padded keys
+    hold NaN."""
+    B, H, Lq, Lk = 6, 8, 700, 333
+    kv = np.array([333, 0, 65, 1, 0, 200], np.int32)
+    w = W.make_custom(B, H, Lq, Lk, d, seed=12, kv_len=kv)
+    nan_bits = np.uint16(0x7FC0)
+    for t in (w.k, w.v, w.k_dot, w.v_dot):
+        for b in range(B):
+            t[b, :, int(kv[b]):] = nan_bits
+    compare(gpu_rows(*run_gpu(w)), oracle_ref(w), f"tile walk d{d}")
