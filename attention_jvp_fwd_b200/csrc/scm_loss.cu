@@ -11,13 +11,19 @@
 // The work is two streaming passes over HBM with one data-dependent scalar
 // between them, so the design is about bandwidth, not arithmetic:
 //   * one thread-block cluster per sample, each CTA a contiguous slice of the
-//     sample; 8 or 16 CTAs per cluster, whichever finishes B samples in
-//     fewer cluster-waves per CTA (the GPU holds fewer 16-CTA clusters);
-//   * pass 1 sums g^2 in fp32; the CTAs meet at a cluster barrier and every
-//     CTA adds the slice sums from distributed shared memory in the same
-//     fixed order, so all hold the same n_b and the result is deterministic;
-//   * pass 2 reads F, F- and g again (g mostly from L2) and writes grad and
-//     the slice sums of r^2, which CTA 0 adds in a fixed order.
+//     sample; the cluster size (1 to 16 CTAs) is the one that finishes B
+//     samples soonest, given how many clusters of each size the GPU holds
+//     at once;
+//   * every thread issues a batch of independent 16-byte loads before it
+//     uses any (16 in pass 1, 8 per tensor in pass 2), so each SM keeps tens
+//     of KB in flight;
+//   * pass 1 sums g^2 in fp32 and reads g with an L2 evict-last hint, so the
+//     second pass finds most of it in L2; the CTAs meet at a cluster barrier
+//     and every CTA adds the slice sums from distributed shared memory in
+//     the same fixed order, so all hold the same n_b and the result is
+//     deterministic;
+//   * pass 2 reads F, F- (evict-first) and g again and writes grad and the
+//     slice sums of r^2, which CTA 0 adds in a fixed order.
 // 16-byte vector loads (8 bf16) when N is a multiple of 8, else bf16 by bf16.
 // No scratch memory: the cross-CTA reduction lives in shared memory.
 
@@ -37,15 +43,19 @@ namespace scml {
 
 using namespace ajvp;
 
-constexpr int THREADS = 512;
+constexpr int THREADS = 256;
 constexpr int MAX_DEVICES = 64;
 
-__device__ __forceinline__ uint4 ld_stream(const void *p)
+constexpr int U1 = 16;  // 16-byte loads in flight per thread, pass 1
+constexpr int U2 = 8;   // per tensor, pass 2
+
+// 16-byte read-only load that skips L1, with an L2 eviction policy.
+__device__ __forceinline__ uint4 ld_stream(const void *p, uint64_t pol)
 {
     uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
+                 : "l"(p), "l"(pol));
     return v;
 }
 
@@ -103,21 +113,47 @@ __global__ void __launch_bounds__(THREADS, 1)
     const long long units = VEC ? N / 8 : N;
     const long long lo = units * rank / ncta, hi = units * (rank + 1) / ncta;
     const size_t base = static_cast<size_t>(b) * static_cast<size_t>(N);
+    const uint4 *fv = reinterpret_cast<const uint4 *>(f + base);
+    const uint4 *ev = reinterpret_cast<const uint4 *>(fe + base);
+    const uint4 *gv = reinterpret_cast<const uint4 *>(g + base);
+    uint4 *dv = grad ? reinterpret_cast<uint4 *>(grad + base) : nullptr;
+    const uint64_t keep = l2_policy_evict_last();
+    const uint64_t once = l2_policy_evict_first();
+    constexpr long long STEP2 = static_cast<long long>(THREADS) * U2;
+
+    // one pass-2 batch: U2 units of F, F- and g per thread
+    uint4 xf[U2], xe[U2], xg[U2];
+    auto load2 = [&](const long long u0) {
+#pragma unroll
+        for (int k = 0; k < U2; ++k) {
+            const long long u = u0 + static_cast<long long>(k) * THREADS;
+            const bool in = u < hi;
+            xf[k] = in ? ld_stream(fv + u, once) : make_uint4(0, 0, 0, 0);
+            xe[k] = in ? ld_stream(ev + u, once) : make_uint4(0, 0, 0, 0);
+            xg[k] = in ? ld_stream(gv + u, once) : make_uint4(0, 0, 0, 0);
+        }
+    };
 
     // ---- pass 1: |g_b|^2
     float acc = 0.f;
     if constexpr (VEC) {
-        const uint4 *gv = reinterpret_cast<const uint4 *>(g + base);
-#pragma unroll 8
-        for (long long u = lo + t; u < hi; u += THREADS) {
-            const uint4 w = ld_stream(gv + u);
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        for (long long u0 = lo + t; u0 < hi; u0 += static_cast<long long>(THREADS) * U1) {
+            uint4 w[U1];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float a0, a1;
-                bf2_to_f(ws[i], a0, a1);
-                acc = fmaf(a0, a0, acc);
-                acc = fmaf(a1, a1, acc);
+            for (int k = 0; k < U1; ++k) {
+                const long long u = u0 + static_cast<long long>(k) * THREADS;
+                w[k] = u < hi ? ld_stream(gv + u, keep) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int k = 0; k < U1; ++k) {
+                const uint32_t ws[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float a0, a1;
+                    bf2_to_f(ws[i], a0, a1);
+                    acc = fmaf(a0, a0, acc);
+                    acc = fmaf(a1, a1, acc);
+                }
             }
         }
     } else {
@@ -134,28 +170,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---- pass 2: r = F - F- - g inv, grad = 2 r, |r|^2
     float acc2 = 0.f;
     if constexpr (VEC) {
-        const uint4 *fv = reinterpret_cast<const uint4 *>(f + base);
-        const uint4 *ev = reinterpret_cast<const uint4 *>(fe + base);
-        const uint4 *gv = reinterpret_cast<const uint4 *>(g + base);
-        uint4 *dv = grad ? reinterpret_cast<uint4 *>(grad + base) : nullptr;
-#pragma unroll 4
-        for (long long u = lo + t; u < hi; u += THREADS) {
-            const uint4 xf = ld_stream(fv + u), xe = ld_stream(ev + u), xg = ld_stream(gv + u);
-            const uint32_t wf[4] = {xf.x, xf.y, xf.z, xf.w}, we[4] = {xe.x, xe.y, xe.z, xe.w},
-                           wg[4] = {xg.x, xg.y, xg.z, xg.w};
-            uint32_t wo[4];
+        for (long long u0 = lo + t; u0 < hi; u0 += STEP2) {
+            load2(u0);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float f0, f1, e0, e1, g0, g1;
-                bf2_to_f(wf[i], f0, f1);
-                bf2_to_f(we[i], e0, e1);
-                bf2_to_f(wg[i], g0, g1);
-                const float r0 = fmaf(-g0, inv, f0 - e0), r1 = fmaf(-g1, inv, f1 - e1);
-                acc2 = fmaf(r0, r0, acc2);
-                acc2 = fmaf(r1, r1, acc2);
-                wo[i] = f_to_bf2(2.f * r0, 2.f * r1);
+            for (int k = 0; k < U2; ++k) {
+                const uint32_t wf[4] = {xf[k].x, xf[k].y, xf[k].z, xf[k].w},
+                               we[4] = {xe[k].x, xe[k].y, xe[k].z, xe[k].w},
+                               wg[4] = {xg[k].x, xg[k].y, xg[k].z, xg[k].w};
+                uint32_t wo[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float f0, f1, e0, e1, g0, g1;
+                    bf2_to_f(wf[i], f0, f1);
+                    bf2_to_f(we[i], e0, e1);
+                    bf2_to_f(wg[i], g0, g1);
+                    const float r0 = fmaf(-g0, inv, f0 - e0), r1 = fmaf(-g1, inv, f1 - e1);
+                    acc2 = fmaf(r0, r0, acc2);
+                    acc2 = fmaf(r1, r1, acc2);
+                    wo[i] = f_to_bf2(2.f * r0, 2.f * r1);
+                }
+                const long long u = u0 + static_cast<long long>(k) * THREADS;
+                if (dv && u < hi) dv[u] = make_uint4(wo[0], wo[1], wo[2], wo[3]);
             }
-            if (dv) dv[u] = make_uint4(wo[0], wo[1], wo[2], wo[3]);
         }
     } else {
         for (long long u = lo + t; u < hi; u += THREADS) {
@@ -193,40 +229,47 @@ static int max_active_clusters(int size)
     return n;
 }
 
-// Resident clusters of 8 and of 16 CTAs on this device (queried once).
+constexpr int MAX_CLUSTER = 16;
+
+// Resident clusters of 1 .. 16 CTAs on this device (queried once; 0 where a
+// size cannot launch).
 template <bool VEC>
-static void cluster_capacity(int dev, int &n8, int &n16)
+static const int *cluster_capacity(int dev)
 {
     static std::mutex mu;
-    static int cap[MAX_DEVICES][2] = {};
+    static int cap[MAX_DEVICES][MAX_CLUSTER + 1] = {};
     static bool done[MAX_DEVICES] = {};
-    n8 = n16 = 0;
-    if (dev < 0 || dev >= MAX_DEVICES) return;
+    static const int none[MAX_CLUSTER + 1] = {};
+    if (dev < 0 || dev >= MAX_DEVICES) return none;
     std::lock_guard<std::mutex> lk(mu);
     if (!done[dev]) {
-        cap[dev][0] = max_active_clusters<VEC>(8);
-        if (cudaFuncSetAttribute(scm_loss_kernel<VEC>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-            cudaSuccess)
-            cap[dev][1] = max_active_clusters<VEC>(16);
+        const bool big = cudaFuncSetAttribute(scm_loss_kernel<VEC>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                              1) == cudaSuccess;
         cudaGetLastError();
+        for (int sz = 1; sz <= MAX_CLUSTER; ++sz) cap[dev][sz] = (sz <= 8 || big) ? max_active_clusters<VEC>(sz) : 0;
         done[dev] = true;
     }
-    n8 = cap[dev][0];
-    n16 = cap[dev][1];
+    return cap[dev];
 }
 
-// Cluster size for B samples: each sample's time scales as 1 / size, and
-// the samples run in ceil(B / resident clusters) waves; take the smaller of
-// waves / size for 8 and 16 CTAs.
+// Cluster size for B samples: a sample's time scales as 1 / size, and the
+// samples run in ceil(B / resident clusters) waves; take the size with the
+// smallest waves / size (the larger size on a tie).
 template <bool VEC>
 static int cluster_size(int dev, int B)
 {
-    int n8, n16;
-    cluster_capacity<VEC>(dev, n8, n16);
-    if (n8 <= 0) return n16 > 0 ? 16 : 0;
-    if (n16 <= 0) return 8;
-    const long long w8 = (B + n8 - 1) / n8, w16 = (B + n16 - 1) / n16;
-    return (w16 * 8 < w8 * 16) ? 16 : 8;  // compare w16 / 16 with w8 / 8
+    const int *cap = cluster_capacity<VEC>(dev);
+    int best = 0;
+    long long bw = 0;  // waves of the best size so far
+    for (int sz = 1; sz <= MAX_CLUSTER; ++sz) {
+        if (cap[sz] <= 0) continue;
+        const long long w = (B + cap[sz] - 1) / cap[sz];
+        if (best == 0 || w * best <= bw * sz) {  // w / sz <= bw / best
+            best = sz;
+            bw = w;
+        }
+    }
+    return best;
 }
 
 static bool overlap(const void *a, size_t na, const void *b, size_t nb)
