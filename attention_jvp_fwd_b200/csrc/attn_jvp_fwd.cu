@@ -71,8 +71,18 @@ enum : int {
     SITE_Q_EMPTY = 12,
 };
 
+// Two ways to split the softmax between its two warpgroups:
+//  - by columns (d = 128): both work on every key tile, warpgroup g on keys
+//    [32g, 32g + 32) of each row, with one running max and one O, O'_acc;
+//  - by tiles (ALT, d = 64): warpgroup g takes the key tiles gg with
+//    gg % 2 == g, whole 64-key rows, and keeps its own running max, l, a and
+//    accumulators O_g, O'_g; the epilogue merges the two.  The two
+//    warpgroups then run out of phase (one's exp2 overlaps the other's
+//    stores), and a row's per-tile latency is spread over two tiles.  The
+//    four accumulators and two S buffers fill TMEM only when d = 64.
 template <int D>
 struct Cfg {
+    static constexpr bool ALT = D == 64;
     static constexpr int NKB = D / 64;               // 128-byte column blocks per row
     static constexpr int NK = (D == 128) ? 3 : 4;    // K ring depth
     static constexpr int NV = (D == 128) ? 2 : 4;    // V ring depth
@@ -87,32 +97,37 @@ struct Cfg {
     static constexpr uint32_t OFF_V = OFF_K + NK * KST_BYTES;
     static constexpr uint32_t OFF_BAR = OFF_V + NV * VST_BYTES;
     // q_full, q_empty, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV],
-    // s_full[2], p_full[2], pd_full[2], o_done, drain
-    static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 1 + 1;
+    // s_full[2], p_full[2], pd_full[2], o_done[2], drain
+    static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 2 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem slot, abort flag
-    // float [640]: per-warpgroup partial l, a ([2][2][128]) and the centring
-    // constant hand-off ([128])
+    // Softmax exchange, floats.  By columns: per-warpgroup partial l, a
+    // ([2][2][128]) and the centring constant hand-off ([128]).  By tiles:
+    // per-warpgroup m, l, a, c ([2][4][128]).
+    static constexpr int XCH_FLOATS = ALT ? 1024 : 640;
     static constexpr uint32_t OFF_XCH = OFF_MISC + 16;
-    static constexpr uint32_t SMEM_BYTES = OFF_XCH + 640 * 4;
+    static constexpr uint32_t SMEM_BYTES = OFF_XCH + XCH_FLOATS * 4;
     // TMEM columns: O | O'_acc | S buffer 0 (S, S'_raw) | S buffer 1.  Both
     // softmax warpgroups read all of S (the row max) but only their own half
     // of S'_raw, columns [BN + 32g, BN + 32g + 32).  Warpgroup g writes its
     // bf16 P (keys 32g..32g+31, two per column) over the first 16 of those
     // columns and P (sS' - c) over the last 16, so no one overwrites a
     // column another warp may still read.
-    static constexpr uint32_t T_O = 0;
-    static constexpr uint32_t T_OD = D;
-    static constexpr uint32_t T_S = 2 * D;
+    //   By tiles the columns are O_0 | O'_0 | O_1 | O'_1 | S buffer 0 | S
+    // buffer 1, and the owner of a buffer writes its bf16 P over S columns
+    // [0, 32) and P (sS' - c) over [32, 64), after it has read all of S.
+    __host__ __device__ static constexpr uint32_t T_O(int g) { return ALT ? g * 2 * D : 0; }
+    __host__ __device__ static constexpr uint32_t T_OD(int g) { return T_O(g) + D; }
+    static constexpr uint32_t T_S = ALT ? 4 * D : 2 * D;
     // column of the bf16 P (pd = false) or P (sS' - c) (pd = true) operand of
     // keys 16kk..16kk+15 inside an S buffer
     __host__ __device__ static constexpr uint32_t t_pk(int kk, bool pd)
     {
-        return BN + (kk >> 1) * 32 + (pd ? 16 : 0) + (kk & 1) * 8;
+        return ALT ? (pd ? 32 : 0) + kk * 8 : BN + (kk >> 1) * 32 + (pd ? 16 : 0) + (kk & 1) * 8;
     }
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, 2 * BN, false);
     static constexpr uint32_t IDESC_SD = idesc_bf16_f32(BM, BN, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
-    static constexpr int P_ARRIVALS = 8;  // one per softmax warp
+    static constexpr int P_ARRIVALS = ALT ? 4 : 8;  // one per softmax warp that writes the tile
     static_assert(T_S + 4 * BN <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -253,8 +268,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
     uint64_t *s_full = v_empty + C::NV;
     uint64_t *p_full = s_full + 2;   // [2] bf16 P written
     uint64_t *pd_full = p_full + 2;  // [2] bf16 P (sS' - c) written
-    uint64_t *o_done = pd_full + 2;  // one phase per key tile: its PV MMAs are done
-    uint64_t *drain = o_done + 1;
+    // [2] the PV MMAs of a key tile are done: by columns o_done[0] has one
+    // phase per key tile; by tiles o_done[g] one per key tile of warpgroup g
+    uint64_t *o_done = pd_full + 2;
+    uint64_t *drain = o_done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -274,7 +291,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             mbar_init(&p_full[s], C::P_ARRIVALS);
             mbar_init(&pd_full[s], C::P_ARRIVALS);
         }
-        mbar_init(o_done, 1);
+        mbar_init(&o_done[0], 1);
+        mbar_init(&o_done[1], 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -427,23 +445,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         // PV of key tile g in two groups: A needs only P (O += P V,
         // O'_acc += P V'), B needs P (sS' - c) as well (O'_acc += P (sS' - c)
         // V), which the softmax writes later; A can then start while B's
-        // operand is formed.  `first`: the query tile's first key tile, which
-        // starts the accumulators.
+        // operand is formed.  `first`: the first key tile of the query tile
+        // for these accumulators, which starts them.  By tiles, key tile gg
+        // goes into warpgroup (gg % 2)'s O_g and O'_g.
         auto issue_pa = [&](const int gk, const bool first) {
             const int s = gk % C::NV;
             tc_fence_after();
             const uint32_t tP = tbase + C::T_S + (gk & 1) * (2 * BN);
+            const int ow = C::ALT ? (gk & 1) : 0;
             const uint64_t dv = sdesc_sw128(smem_addr(smem + C::OFF_V + s * C::VST_BYTES), LBO, 1024);
             const uint64_t dvd = desc_add(dv, C::VHALF_BYTES);
             (void)dvd;
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)  // O += P V
-                mma_ts(tbase + C::T_O, tP + C::t_pk(kk, false), desc_add(dv, kk * 2048), C::IDESC_PV,
+                mma_ts(tbase + C::T_O(ow), tP + C::t_pk(kk, false), desc_add(dv, kk * 2048), C::IDESC_PV,
                        (!first || kk > 0) ? 1u : 0u);
             if constexpr (!ZKV) {
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)  // O'_acc += P V'
-                    mma_ts(tbase + C::T_OD, tP + C::t_pk(kk, false), desc_add(dvd, kk * 2048), C::IDESC_PV,
+                    mma_ts(tbase + C::T_OD(ow), tP + C::t_pk(kk, false), desc_add(dvd, kk * 2048), C::IDESC_PV,
                            (!first || kk > 0) ? 1u : 0u);
             }
         };
@@ -451,13 +471,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const int s = gk % C::NV;
             tc_fence_after();
             const uint32_t tP = tbase + C::T_S + (gk & 1) * (2 * BN);
+            const int ow = C::ALT ? (gk & 1) : 0;
             const uint64_t dv = sdesc_sw128(smem_addr(smem + C::OFF_V + s * C::VST_BYTES), LBO, 1024);
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)  // O'_acc += P(sS' - c) V (with V' = 0 it starts O'_acc)
-                mma_ts(tbase + C::T_OD, tP + C::t_pk(kk, true), desc_add(dv, kk * 2048), C::IDESC_PV,
+                mma_ts(tbase + C::T_OD(ow), tP + C::t_pk(kk, true), desc_add(dv, kk * 2048), C::IDESC_PV,
                        (!ZKV || !first || kk > 0) ? 1u : 0u);
             mma_commit(&v_empty[s]);
-            mma_commit(o_done);
+            mma_commit(&o_done[ow]);
         };
         // Fixed order per query tile: S_0, S_1, PV_0, S_2, PV_1, ...: S_{j+1}
         // runs on the tensor core while the softmax works on key tile j, and
@@ -489,10 +510,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 ok = wait_u(&v_full[gk % C::NV], (gk / C::NV) & 1, SITE_V_FULL);
                 if (ok) ok = wait_u(&p_full[gk & 1], (gk >> 1) & 1, SITE_P_FULL);
                 if (!ok) break;
-                issue_pa(gk, j == 0);
+                const bool first = C::ALT ? j < 2 : j == 0;
+                issue_pa(gk, first);
                 ok = wait_u(&pd_full[gk & 1], (gk >> 1) & 1, SITE_P_FULL);
                 if (!ok) break;
-                issue_pb(gk, j == 0);
+                issue_pb(gk, first);
             }
             gg += t.nT;
         }
@@ -503,22 +525,305 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        // Two warpgroups, thread = query row.  Warpgroup g owns key columns
-        // [32g, 32g + 32) of every key tile; at the end of a query tile it
+        // Two warpgroups, thread = query row.  By columns, warpgroup g owns
+        // key columns [32g, 32g + 32) of every key tile; by tiles, the key
+        // tiles gg with gg % 2 == g.  At the end of a query tile warpgroup g
         // writes output g (0: O and lse, 1: O' and lse').
         const int g = (warp - 2) >> 2;
         const int quad = warp & 3;  // TMEM lane quadrant this warp may touch
         const int r = quad * 32 + lane;
         const int gt = tid - 64 - g * 128;  // thread index inside the warpgroup
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-        // [0, 512): per-warpgroup l and a of the query tile ([slot][g][row]);
-        // [512, 640): the centring constant handed from warpgroup 0 to 1.
-        // The hand-off has a slot of its own, because warpgroup 0 may start
-        // the next query tile while warpgroup 1 still reads the l, a of this one.
         float *xch = reinterpret_cast<float *>(smem + C::OFF_XCH);
         const float sl2 = p.sl2;
         const float sc = p.scale;
         const bool neg = sl2 < 0.f;
+        if constexpr (C::ALT) {
+            int gg = 0;
+            const uint32_t tS = tbase + lane_off + C::T_S + g * (2 * BN);  // this warpgroup's S buffer
+            for (int w = blockIdx.x; w < p.n_tiles; w += gridDim.x) {
+                const Tile t = tile_of(p, w);
+                const int grow = t.q0 + r;
+                __nv_bfloat16 *out_ptr =
+                    static_cast<__nv_bfloat16 *>(g == 0 ? p.o : p.od) + (static_cast<size_t>(t.bh) * p.Lq + grow) * D;
+                const size_t lrow = static_cast<size_t>(t.bh) * p.Lq + grow;
+                if (t.nT == 0) {
+                    if (grow < p.Lq) {
+                        const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                        for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4 *>(out_ptr)[c] = z;
+                        if (g == 0) p.lse[lrow] = -INFINITY;
+                        if (g == 1 && p.lse_dot) p.lse_dot[lrow] = 0.f;
+                    }
+                    continue;
+                }
+                const int nb = t.nb, nT = t.nT;
+                // this warpgroup's running max (log2 units), l, a and centring
+                // constant over its own key tiles
+                float m_used = -INFINITY, l = 0.f, acc_a = 0.f, cctr = 0.f;
+                bool err = false;
+                int nown = 0, last = 0;
+                for (int j = ((gg & 1) == g) ? 0 : 1; j < nT; j += 2) {
+                    const int gk = gg + j;
+                    if (!__all_sync(0xffffffffu, wait_bar_fast(&s_full[g], (gk >> 1) & 1, wc, SITE_S_FULL))) {
+                        err = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int vt = nb - j * BN;  // valid keys in the tile
+                    const bool tail = vt < BN;
+                    uint32_t ra[32], rb[32];
+                    tmem_ld32(tS, ra);       // S, keys 0..31
+                    tmem_ld32(tS + 32, rb);  // S, keys 32..63
+                    tmem_ld_wait2(ra, rb);
+                    if (tail) {
+                        const float pad = neg ? INFINITY : -INFINITY;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            ra[i] = (i < vt) ? ra[i] : f2u(pad);
+                            rb[i] = (i + 32 < vt) ? rb[i] : f2u(pad);
+                        }
+                    }
+                    const float mx = neg ? row_min64(ra, rb) : row_max64(ra, rb);
+                    uint32_t rd[32];
+                    tmem_ld32(tS + BN, rd);  // S'_raw, keys 0..31 (waited for below)
+                    const float m_tile = mx * sl2;
+                    float alpha = 1.f;
+                    bool rescale = false;
+                    if (nown == 0) {
+                        m_used = m_tile;
+                    } else if (m_tile > m_used + RESCALE_THRESHOLD) {
+                        alpha = ex2_approx(m_used - m_tile);
+                        m_used = m_tile;
+                        rescale = true;
+                    }
+                    l *= alpha;
+                    acc_a *= alpha;
+                    float x[64];
+                    {
+                        const uint64_t sl22 = f2_pack(sl2, sl2);
+                        const uint64_t nm2 = f2_pack(-m_used, -m_used);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float t0, t1, t2, t3;
+                            f2_unpack(f2_fma(f2_pack(u2f(ra[2 * i]), u2f(ra[2 * i + 1])), sl22, nm2), t0, t1);
+                            f2_unpack(f2_fma(f2_pack(u2f(rb[2 * i]), u2f(rb[2 * i + 1])), sl22, nm2), t2, t3);
+                            x[2 * i] = ex2_approx(t0);
+                            x[2 * i + 1] = ex2_approx(t1);
+                            x[32 + 2 * i] = ex2_approx(t2);
+                            x[33 + 2 * i] = ex2_approx(t3);
+                        }
+                    }
+                    if (tail) {
+                        // padded keys: p = 0 exactly (the pad times a zero scale is NaN)
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) x[i] = (i < vt) ? x[i] : 0.f;
+                    }
+                    {
+                        uint64_t s0 = f2_pack(x[0], x[1]), s1 = f2_pack(x[2], x[3]);
+                        uint64_t s2 = f2_pack(x[32], x[33]), s3 = f2_pack(x[34], x[35]);
+#pragma unroll
+                        for (int i = 2; i < 16; i += 2) {
+                            s0 = f2_add(s0, f2_pack(x[2 * i], x[2 * i + 1]));
+                            s1 = f2_add(s1, f2_pack(x[2 * i + 2], x[2 * i + 3]));
+                            s2 = f2_add(s2, f2_pack(x[32 + 2 * i], x[33 + 2 * i]));
+                            s3 = f2_add(s3, f2_pack(x[34 + 2 * i], x[35 + 2 * i]));
+                        }
+                        float u0, u1, u2, u3;
+                        f2_unpack(f2_add(s0, s2), u0, u1);
+                        f2_unpack(f2_add(s1, s3), u2, u3);
+                        l += (u0 + u1) + (u2 + u3);
+                    }
+                    if (nown >= 1) {
+                        // PV of this warpgroup's previous key tile must be done
+                        // before O_g may be rescaled (it always is by now: its
+                        // o_done phase precedes this tile's S)
+                        if (!__all_sync(0xffffffffu,
+                                        wait_bar_fast(&o_done[g], ((gk >> 1) - 1) & 1, wc, SITE_O_DONE))) {
+                            err = true;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+                        for (int c = 0; c < 2 * D; c += 32) {  // O_g then O'_g
+                            uint32_t tt[32];
+                            tmem_ld32(tbase + lane_off + C::T_O(g) + c, tt);
+                            tmem_ld_wait(tt);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) tt[i] = f2u(u2f(tt[i]) * alpha);
+                            tmem_st32(tbase + lane_off + C::T_O(g) + c, tt);
+                        }
+                    }
+                    if (tail) {
+                        // Zero the V (and V') rows of padded keys so their bits
+                        // (NaN included) cannot reach the PV products.
+                        const int s = gk % C::NV;
+                        if (!__all_sync(0xffffffffu, wait_bar(&v_full[s], (gk / C::NV) & 1, wc, SITE_V_TAIL))) {
+                            err = true;
+                            break;
+                        }
+                        uint8_t *vst = smem + C::OFF_V + s * C::VST_BYTES;
+                        const int per_blk = (BN - vt) * 8;  // 16-byte chunks per 64-column block
+                        const int chunks = (ZKV ? 1 : 2) * C::NKB * per_blk;
+                        for (int idx = gt; idx < chunks; idx += 128) {
+                            const int blk = idx / per_blk;  // V blocks, then V' blocks
+                            const int rem = idx - blk * per_blk;
+                            *reinterpret_cast<uint4 *>(vst + blk * (BN * 128) + (vt + (rem >> 3)) * 128 +
+                                                       (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    {
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+                        tmem_st32(tS, pk);  // P over S columns [0, 32): S has been read
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&p_full[g]);
+                    // ---- bf16 P (s S' - c) while the tensor core multiplies P
+                    tmem_ld_wait(rd);
+                    if (nown == 0) {
+                        // centring constant c: the p-weighted mean of s S' over
+                        // keys 0..31 of this warpgroup's first key tile (key 0
+                        // is always valid)
+                        float n0 = 0.f, n1 = 0.f, w0 = 0.f, w1 = 0.f;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            n0 += (tail && i >= vt) ? 0.f : x[i] * (u2f(rd[i]) * sc);
+                            n1 += (tail && i + 1 >= vt) ? 0.f : x[i + 1] * (u2f(rd[i + 1]) * sc);
+                            w0 += x[i];
+                            w1 += x[i + 1];
+                        }
+                        cctr = (n0 + n1) / (w0 + w1);
+                    }
+                    uint32_t re[32];
+                    tmem_ld32(tS + BN + 32, re);  // S'_raw, keys 32..63
+                    const uint64_t sc2 = f2_pack(sc, sc);
+                    const uint64_t nc2 = f2_pack(-cctr, -cctr);
+                    uint64_t a0 = 0, a1 = 0;
+                    // keys [32h, 32h + 32) from v (S'_raw) into TMEM column 32 + 16h
+                    auto pd_half = [&](const uint32_t (&v)[32], const int h) {
+                        uint32_t pdk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int k0 = 32 * h + 2 * i;
+                            const uint64_t p2 = f2_pack(x[k0], x[k0 + 1]);
+                            const uint64_t d2 = f2_mul(f2_fma(f2_pack(u2f(v[2 * i]), u2f(v[2 * i + 1])), sc2, nc2), p2);
+                            float d0, d1;
+                            f2_unpack(d2, d0, d1);
+                            if (tail) {
+                                d0 = (k0 < vt) ? d0 : 0.f;
+                                d1 = (k0 + 1 < vt) ? d1 : 0.f;
+                            }
+                            pdk[i] = pack_bf16x2(d0, d1);
+                            // the two rounded values as fp32
+                            const uint64_t r2 = f2_pack(u2f(pdk[i] << 16), u2f(pdk[i] & 0xFFFF0000u));
+                            if (i & 1) a1 = f2_add(a1, r2);
+                            else a0 = f2_add(a0, r2);
+                        }
+                        tmem_st16(tS + 32 + 16 * h, pdk);
+                    };
+                    pd_half(rd, 0);
+                    tmem_ld_wait(re);
+                    pd_half(re, 1);
+                    {
+                        float u0, u1, u2, u3;
+                        f2_unpack(a0, u0, u1);
+                        f2_unpack(a1, u2, u3);
+                        acc_a += (u0 + u1) + (u2 + u3);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pd_full[g]);
+                    ++nown;
+                    last = gk;
+                }
+                bool ok;
+                {
+                    bool done = !err;
+                    if (!err && nown > 0) done = wait_bar(&o_done[g], (last >> 1) & 1, wc, SITE_O_DONE, true);
+                    ok = bar_and(BAR_SOFT, NSOFT, done);  // reached by all 256 threads
+                }
+                // whether warpgroup h had key tiles in this query tile (the same
+                // for every thread, so the TMEM loads below stay warp-uniform)
+                const bool has0 = nT >= 2 || (gg & 1) == 0;
+                const bool has1 = nT >= 2 || (gg & 1) == 1;
+                gg += nT;
+                if (!ok) break;
+                tc_fence_after();
+                // Merge the two warpgroups' partial softmaxes.  With
+                // M = max(m_0, m_1), b_h = 2^(m_h - M), L = sum_h b_h l_h:
+                //   O   = sum_h b_h O_h / L,
+                //   lse' = mu = sum_h b_h (a_h + c_h l_h) / L,
+                //   O'  = sum_h b_h (O'_h + (c_h - mu) O_h) / L.
+                xch[(g * 4 + 0) * 128 + r] = m_used;
+                xch[(g * 4 + 1) * 128 + r] = l;
+                xch[(g * 4 + 2) * 128 + r] = acc_a;
+                xch[(g * 4 + 3) * 128 + r] = cctr;
+                bar_sync(BAR_SOFT, NSOFT);
+                const float m0 = xch[r], l0 = xch[128 + r], a0v = xch[256 + r], c0v = xch[384 + r];
+                const float m1 = xch[512 + r], l1 = xch[640 + r], a1v = xch[768 + r], c1v = xch[896 + r];
+                const float M = has0 ? (has1 ? fmaxf(m0, m1) : m0) : m1;
+                const float b0 = has0 ? ex2_approx(m0 - M) : 0.f;
+                const float b1 = has1 ? ex2_approx(m1 - M) : 0.f;
+                const float lt = (has0 ? b0 * l0 : 0.f) + (has1 ? b1 * l1 : 0.f);
+                const float inv_l = 1.f / lt;
+                const float mu = ((has0 ? b0 * fmaf(c0v, l0, a0v) : 0.f) + (has1 ? b1 * fmaf(c1v, l1, a1v) : 0.f)) * inv_l;
+                const float w0 = b0 * inv_l, w1 = b1 * inv_l;
+                const float k0 = w0 * (c0v - mu), k1 = w1 * (c1v - mu);
+#pragma unroll 1
+                for (int c = 0; c < D; c += 32) {
+                    float acc[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (!(h == 0 ? has0 : has1)) continue;
+                        const float wh = h == 0 ? w0 : w1, kh = h == 0 ? k0 : k1;
+                        uint32_t ov[32];
+                        tmem_ld32(tbase + lane_off + C::T_O(h) + c, ov);
+                        if (g == 0) {
+                            tmem_ld_wait(ov);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) acc[i] = fmaf(wh, u2f(ov[i]), acc[i]);
+                        } else {
+                            uint32_t odv[32];
+                            tmem_ld32(tbase + lane_off + C::T_OD(h) + c, odv);
+                            tmem_ld_wait2(ov, odv);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) acc[i] = fmaf(wh, u2f(odv[i]), fmaf(kh, u2f(ov[i]), acc[i]));
+                        }
+                    }
+                    if (grow < p.Lq) {
+                        uint32_t pv[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+                        uint4 *dst = reinterpret_cast<uint4 *>(out_ptr + c);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pv[4 * i], pv[4 * i + 1], pv[4 * i + 2], pv[4 * i + 3]);
+                    }
+                }
+                if (g == 0 && grow < p.Lq) p.lse[lrow] = (M + log2f(lt)) * 0.69314718055994531f;
+                if (g == 1 && p.lse_dot && grow < p.Lq) p.lse_dot[lrow] = mu;
+                // Both warpgroups read O_0 and O_1 above; the next query tile's
+                // first P (after which the MMAs restart an accumulator) comes
+                // from one warpgroup only, so meet here first.  This also
+                // keeps the exchange slots from being overwritten early.
+                tc_fence_before();
+                bar_sync(BAR_SOFT, NSOFT);
+            }
+        } else {
+        // [0, 512): per-warpgroup l and a of the query tile ([slot][g][row]);
+        // [512, 640): the centring constant handed from warpgroup 0 to 1.
+        // The hand-off has a slot of its own, because warpgroup 0 may start
+        // the next query tile while warpgroup 1 still reads the l, a of this one.
         const int c0 = 32 * g;
         int gg = 0;
         for (int w = blockIdx.x; w < p.n_tiles; w += gridDim.x) {
@@ -655,14 +960,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     // PV of the previous key tile must be done before O may be
                     // rescaled; every warp observes every phase of o_done in
                     // order (phase gk needs this warp's P of key tile gk).
-                    if (!__all_sync(0xffffffffu, wait_bar_fast(o_done, (gk - 1) & 1, wc, SITE_O_DONE))) {
+                    if (!__all_sync(0xffffffffu, wait_bar_fast(&o_done[0], (gk - 1) & 1, wc, SITE_O_DONE))) {
                         err = true;
                         break;
                     }
                     tc_fence_after();
                 }
                 if (__any_sync(0xffffffffu, rescale)) {
-                    const uint32_t tacc = tbase + lane_off + (g == 0 ? C::T_O : C::T_OD);
+                    const uint32_t tacc = tbase + lane_off + (g == 0 ? C::T_O(0) : C::T_OD(0));
 #pragma unroll 1
                     for (int c = 0; c < D; c += 32) {
                         uint32_t tt[32];
@@ -737,7 +1042,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             bool ok;
             {
                 bool done = false;
-                if (!err) done = wait_bar(o_done, (gg + nT - 1) & 1, wc, SITE_O_DONE, true);
+                if (!err) done = wait_bar(&o_done[0], (gg + nT - 1) & 1, wc, SITE_O_DONE, true);
                 ok = bar_and(BAR_SOFT, NSOFT, done);  // reached by all 256 threads
             }
             gg += nT;
@@ -751,8 +1056,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const float lt = xch[r] + xch[128 + r];
             const float inv_l = 1.f / lt;
             const float coef = (xch[256 + r] + xch[384 + r]) * inv_l;
-            const uint32_t to = tbase + lane_off + C::T_O;
-            const uint32_t tod = tbase + lane_off + C::T_OD;
+            const uint32_t to = tbase + lane_off + C::T_O(0);
+            const uint32_t tod = tbase + lane_off + C::T_OD(0);
 #pragma unroll 1
             for (int c = 0; c < D; c += 32) {
                 uint32_t ov[32], odv[32];
@@ -785,6 +1090,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             // the next query tile's first P (which lets the MMAs restart O and
             // O'_acc) is signalled after a tcgen05 fence that orders these loads
         }
+        }  // by columns
     }
 
     tc_fence_before();
