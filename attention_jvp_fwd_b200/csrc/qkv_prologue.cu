@@ -15,16 +15,21 @@
 // and writes q, k, v, q', k', v' in the attention layout [B, H, L, d], so
 // the attention kernel reads them directly.
 //
-// A tile is 128 tokens x one head: two tcgen05 GEMMs that share the weight
-// tile, Y = X W_h^T and Y' = X' W_h^T (M = 128, N = d, K = D), both
-// accumulating in TMEM.  The kernel is persistent (one CTA per SM walks the
-// tiles) with two accumulator sets, so the epilogue of one tile overlaps the
-// MMAs of the next.  A TMA warp streams X, X' and W_h in 64-column slices
-// through a 4-stage ring that runs on across tiles; one warp issues the
-// MMAs; four epilogue warps (thread = token) reduce each row's y^2 and y y'
-// over the head, apply the RMSNorm and its tangent, and store bf16.  Waits
-// are bounded like the attention kernel's (status word read by
-// qkv_prologue_check).
+// A tile is 256 tokens x one head, owned by a cluster of two CTAs (a CTA
+// pair): two tcgen05 GEMMs that share the weight tile, Y = X W_h^T and
+// Y' = X' W_h^T (M = 256, N = d, K = D), issued by the leader CTA as
+// cta_group::2 MMAs.  Each CTA stages its own 128 tokens of X and X' and half
+// of the rows of W_h, and receives Y, Y' of its own tokens in its TMEM, so
+// each CTA reads only half of the weight slice from shared memory per MMA
+// (the single-CTA form of this kernel was bound by shared-memory bandwidth).
+// The kernel is persistent (one pair per two SMs walks the tiles) with two
+// accumulator sets, so the epilogue of one tile overlaps the MMAs of the
+// next.  In each CTA a TMA warp streams X, X' and its half of W_h in
+// 64-column slices through a 5-stage ring that runs on across tiles; the
+// leader's MMA warp issues the MMAs; four epilogue warps (thread = token)
+// reduce each row's y^2 and y y' over the head, apply the RMSNorm and its
+// tangent, and store bf16.  Waits are bounded like the attention kernel's
+// (status word read by qkv_prologue_check).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -44,23 +49,23 @@ namespace qkvp {
 
 using namespace ajvp;
 
-constexpr int BM = 128;   // tokens per tile (TMEM lanes)
+constexpr int BM = 128;   // tokens per CTA per tile (TMEM lanes); a pair covers 2 BM
 constexpr int BK = 64;    // D columns per stage (one 128-byte swizzle row)
-constexpr int NS = 4;     // ring stages
+constexpr int NS = 5;     // ring stages
 constexpr int NTHREADS = 192;  // TMA warp, MMA warp, 4 epilogue warps
 constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 
 template <int DH>
 struct PCfg {
-    static constexpr uint32_t A_BYTES = BM * BK * 2;   // one of X, X' per stage
-    static constexpr uint32_t B_BYTES = DH * BK * 2;   // W_h slice per stage
+    static constexpr uint32_t A_BYTES = BM * BK * 2;         // one of X, X' per stage
+    static constexpr uint32_t B_BYTES = (DH / 2) * BK * 2;   // this CTA's half of the W_h slice
     static constexpr uint32_t ST_BYTES = 2 * A_BYTES + B_BYTES;
     static constexpr uint32_t OFF_BAR = NS * ST_BYTES;
     static constexpr uint32_t OFF_MISC = OFF_BAR + (2 * NS + 5) * 8;  // tmem slot, abort
     static constexpr uint32_t OFF_GAMMA = OFF_MISC + 16;              // float [2][DH]
     static constexpr uint32_t SMEM_BYTES = OFF_GAMMA + 2 * DH * 4;
     static constexpr uint32_t TMEM_COLS = 4 * DH;                      // two sets of Y | Y'
-    static constexpr uint32_t IDESC = idesc_bf16_f32(BM, DH, false);
+    static constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, DH, false);  // M = 256 over the pair
     static_assert(SMEM_BYTES + 1024 <= 232448, "shared memory budget");
 };
 
@@ -68,25 +73,27 @@ struct Params {
     CUtensorMap tm_x, tm_xd, tm_w;
     const float *gamma_q, *gamma_k;
     __nv_bfloat16 *out[6];  // q, k, v, q', k', v'
-    int T, L, H, D, tiles_m;
+    int T, L, H, D, tiles_m;  // tiles_m: 256-token blocks
     float eps;
     uint64_t timeout_ns;
 };
 
 __device__ int g_status;
 
-// Bounded wait; gives up when another role has aborted (if honor_abort) or
-// after `limit` ns (then it records `site` and aborts the CTA itself).
+// Bounded wait (acquire at cluster scope: most of these barriers are
+// signalled from the other CTA of the pair); gives up when another role has
+// aborted (if honor_abort) or after `limit` ns (then it records `site` and
+// aborts the CTA itself).
 __device__ __noinline__ bool wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint64_t limit, int site,
                                   bool honor_abort = true)
 {
     const uint32_t a = smem_addr(bar);
-    if (mbar_try_wait(a, parity)) return true;
+    if (mbar_try_wait_cluster(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(a, parity)) return true;
+            if (mbar_try_wait_cluster(a, parity)) return true;
         if (honor_abort && *abort) return false;
         if (globaltimer_ns() - t0 > limit) {
             *abort = 1;
@@ -104,17 +111,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
     // 128-byte swizzle atoms want 1024-byte alignment
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();  // 0: the leader, which issues the MMAs
+    const bool leader = rank == 0;
     const int tiles_n = 3 * p.H;
     const int n_tiles = p.tiles_m * tiles_n;
     const int nk = p.D / BK;
-    // this CTA's tiles: blockIdx.x, + gridDim.x, ...  (head tile fastest, so
-    // CTAs running together share the token tile through L2)
-    const int my_tiles = blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    // this pair's tiles: cl, cl + ncl, ...  (head tile fastest, so pairs
+    // running together share the token tile through L2)
+    const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+    const int my_tiles = cl < n_tiles ? (n_tiles - 1 - cl) / ncl + 1 : 0;
 
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *empty = full + NS;
-    uint64_t *acc_full = empty + NS;  // [2] accumulator set b holds a finished tile
-    uint64_t *acc_empty = acc_full + 2;  // [2] the epilogue has read accumulator set b
+    // full, acc_empty and drain are used in the leader only; empty and
+    // acc_full in both CTAs (the leader's commits reach both)
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);  // [NS] both CTAs' slices landed
+    uint64_t *empty = full + NS;         // [NS] the MMAs are done with this CTA's slice
+    uint64_t *acc_full = empty + NS;     // [2] accumulator set b holds a finished tile
+    uint64_t *acc_empty = acc_full + 2;  // [2] both epilogues have read accumulator set b
     uint64_t *drain = acc_empty + 2;     // MMAs in flight after an abort are done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
@@ -127,33 +139,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+            mbar_init(&acc_empty[b], 8);  // one arrival per epilogue warp of each CTA
         }
         mbar_init(drain, 1);
         *abort = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish_pair();
     }
     if (warp >= 2) {
         for (int i = tid - 64; i < 2 * DH; i += 128) gamma[i] = i < DH ? p.gamma_q[i] : p.gamma_k[i - DH];
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
+    const uint32_t full_lead = mapa_shared(smem_addr(full), 0);
+    const uint32_t acc_empty_lead = mapa_shared(smem_addr(acc_empty), 0);
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA: one ring across all tiles
+        // Both CTAs' slices complete on the leader's full barrier; the
+        // leader announces the bytes of both.
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_last();
             long long issued = 0;  // slices loaded so far
             bool ok = true;
             for (int li = 0; li < my_tiles && ok; ++li) {
-                const int t = blockIdx.x + li * gridDim.x;
+                const int t = cl + li * ncl;
                 const int nt = t % tiles_n, mt = t / tiles_n;
+                const int row = mt * 2 * BM + static_cast<int>(rank) * BM;
+                const int wrow = nt * DH + static_cast<int>(rank) * (DH / 2);
                 for (int k = 0; k < nk; ++k) {
                     const int s = static_cast<int>(issued % NS);
                     if (issued >= NS &&
@@ -162,60 +180,68 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
                         break;
                     }
                     uint8_t *st = smem + s * C::ST_BYTES;
-                    mbar_arrive_expect_tx(&full[s], C::ST_BYTES);
-                    tma_load_3d(st, &p.tm_x, &full[s], k * BK, mt * BM, 0, pol);
-                    tma_load_3d(st + C::A_BYTES, &p.tm_xd, &full[s], k * BK, mt * BM, 0, pol);
-                    tma_load_3d(st + 2 * C::A_BYTES, &p.tm_w, &full[s], k * BK, nt * DH, 0, pol);
+                    const uint32_t fb = full_lead + s * 8;
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::ST_BYTES);
+                    tma_load_3d_pair(st, &p.tm_x, fb, k * BK, row, 0, pol);
+                    tma_load_3d_pair(st + C::A_BYTES, &p.tm_xd, fb, k * BK, row, 0, pol);
+                    tma_load_3d_pair(st + 2 * C::A_BYTES, &p.tm_w, fb, k * BK, wrow, 0, pol);
                     ++issued;
                 }
             }
-            // let every load issued land before the CTA can exit (the last
-            // phase of each stage, so the parity test is unambiguous)
-            for (long long q = (issued > NS ? issued - NS : 0); q < issued; ++q)
-                wait(&full[q % NS], static_cast<uint32_t>(q / NS) & 1, abort, p.timeout_ns, 2, false);
+            // let every load issued land before the CTAs can exit: the
+            // leader waits for the last phase of each stage (the peer's
+            // loads complete on the same barriers; the final cluster barrier
+            // keeps the peer alive until then)
+            if (leader)
+                for (long long q = (issued > NS ? issued - NS : 0); q < issued; ++q)
+                    wait(&full[q % NS], static_cast<uint32_t>(q / NS) & 1, abort, p.timeout_ns, 2, false);
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA (warp-wide, elected lane)
-        bool ok = true, issued = false;
-        long long used = 0;  // slices consumed so far
-        for (int li = 0; li < my_tiles && ok; ++li) {
-            const int b = li & 1;
-            const uint32_t acc = tbase + b * (2 * DH);
-            if (li >= 2) {
-                ok = __all_sync(0xffffffffu, wait(&acc_empty[b], ((li >> 1) - 1) & 1, abort, p.timeout_ns, 6));
-                if (!ok) break;
-                tc_fence_after();
-            }
-            for (int k = 0; k < nk; ++k, ++used) {
-                const int s = static_cast<int>(used % NS);
-                ok = __all_sync(0xffffffffu, wait(&full[s], static_cast<uint32_t>(used / NS) & 1, abort,
-                                                  p.timeout_ns, 3));
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t st = smem_addr(smem + s * C::ST_BYTES);
-                const uint64_t dx = sdesc_sw128(st, 16, 1024);
-                const uint64_t dxd = sdesc_sw128(st + C::A_BYTES, 16, 1024);
-                const uint64_t dw = sdesc_sw128(st + 2 * C::A_BYTES, 16, 1024);
+        // ---------------------------------------------------------------- MMA (leader; warp-wide, elected lane)
+        if (leader) {
+            bool ok = true, issued = false;
+            long long used = 0;  // slices consumed so far
+            for (int li = 0; li < my_tiles && ok; ++li) {
+                const int b = li & 1;
+                const uint32_t acc = tbase + b * (2 * DH);
+                if (li >= 2) {
+                    ok = __all_sync(0xffffffffu, wait(&acc_empty[b], ((li >> 1) - 1) & 1, abort, p.timeout_ns, 6));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                for (int k = 0; k < nk; ++k, ++used) {
+                    const int s = static_cast<int>(used % NS);
+                    ok = __all_sync(0xffffffffu, wait(&full[s], static_cast<uint32_t>(used / NS) & 1, abort,
+                                                      p.timeout_ns, 3));
+                    if (!ok) break;
+                    tc_fence_after();
+                    // the same shared-memory offsets in both CTAs: A rows 0-127
+                    // and B rows 0 .. d/2-1 here, the rest in the peer
+                    const uint32_t st = smem_addr(smem + s * C::ST_BYTES);
+                    const uint64_t dx = sdesc_sw128(st, 16, 1024);
+                    const uint64_t dxd = sdesc_sw128(st + C::A_BYTES, 16, 1024);
+                    const uint64_t dw = sdesc_sw128(st + 2 * C::A_BYTES, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    mma_ss(acc, desc_add(dx, kk * 32), desc_add(dw, kk * 32), C::IDESC,
-                           (k > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_ss_pair(acc, desc_add(dx, kk * 32), desc_add(dw, kk * 32), C::IDESC,
+                                    (k > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    mma_ss(acc + DH, desc_add(dxd, kk * 32), desc_add(dw, kk * 32), C::IDESC,
-                           (k > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&empty[s]);
-                issued = true;
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_ss_pair(acc + DH, desc_add(dxd, kk * 32), desc_add(dw, kk * 32), C::IDESC,
+                                    (k > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit_pair_mc(&empty[s], 0x3);
+                    issued = true;
+                }
+                if (!ok) break;
+                mma_commit_pair_mc(&acc_full[b], 0x3);
             }
-            if (!ok) break;
-            mma_commit(&acc_full[b]);
-        }
-        if (!ok && issued) {
-            // nobody else waits for the MMAs in flight after an abort: drain
-            // them here, so TMEM is not freed under them
-            mma_commit(drain);
-            wait(drain, 0, abort, p.timeout_ns, 5, false);
+            if (!ok && issued) {
+                // nobody else waits for the MMAs in flight after an abort:
+                // drain them here, so TMEM is not freed under them
+                mma_commit_pair_mc(drain, 0x1);
+                wait(drain, 0, abort, p.timeout_ns, 5, false);
+            }
         }
         __syncwarp();
     } else {
@@ -225,7 +251,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         for (int li = 0; li < my_tiles; ++li) {
             const int b = li & 1;
-            const int t_idx = blockIdx.x + li * gridDim.x;
+            const int t_idx = cl + li * ncl;
             const int nt = t_idx % tiles_n, mt = t_idx / tiles_n;
             const int part = nt / p.H, head = nt % p.H;
             const uint32_t ty = tbase + lane_off + b * (2 * DH), tyd = ty + DH;
@@ -233,7 +259,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
             ok = __all_sync(0xffffffffu, ok && !*abort);  // warp-uniform: tcgen05.ld below is collective
             if (!ok) break;
             tc_fence_after();
-            const int t = mt * BM + r;
+            const int t = mt * 2 * BM + static_cast<int>(rank) * BM + r;
             const float *g = gamma + (part == 1 ? DH : 0);
             float rs = 1.f, mix = 0.f;
             if (part < 2) {
@@ -271,10 +297,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
                 tmem_ld_wait2(a, e);
                 if (c + 32 == DH) {
                     // the last read of this accumulator set: hand it back to
-                    // the MMA warp before the stores
+                    // the leader's MMA warp before the stores
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&acc_empty[b]);
+                    if (lane == 0) mbar_arrive_cluster(acc_empty_lead + b * 8);
                 }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -306,10 +332,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) qkv_prologue_kernel(const __grid_
         }
     }
     tc_fence_before();
-    __syncthreads();
+    // neither CTA leaves while the leader's MMAs may still read the peer's
+    // shared memory or write its TMEM, or loads may still signal the leader
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tbase, C::TMEM_COLS);
+        tmem_dealloc_pair(tbase, C::TMEM_COLS);
     }
 }
 
@@ -351,24 +379,61 @@ static bool make_map(CUtensorMap *m, const void *base, long long rows, int cols,
 
 constexpr int MAX_DEVICES = 64;
 
+// Launch configuration of the pair kernel (grid = 2 x pairs, clusters of 2).
 template <int DH>
-static int launch_kernel(const Params &prm, long long grid, cudaStream_t s)
+static void pair_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, unsigned pairs, cudaStream_t s)
+{
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(NTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = PCfg<DH>::SMEM_BYTES + 1024;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+}
+
+// Per device, once: the shared-memory opt-in and how many CTA pairs fit on
+// the GPU at once (a persistent grid must not spill into a second wave).
+template <int DH>
+static int resident_pairs(int dev)
 {
     static std::mutex mu;
-    static bool done[MAX_DEVICES] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return ATTN_JVP_ERR_LAUNCH;
-    const int smem = static_cast<int>(PCfg<DH>::SMEM_BYTES + 1024);
-    {
-        std::lock_guard<std::mutex> g(mu);
-        if (!done[dev]) {
-            if (cudaFuncSetAttribute(qkv_prologue_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-                cudaSuccess)
-                return ATTN_JVP_ERR_LAUNCH;
-            done[dev] = true;
+    static int pairs[MAX_DEVICES] = {};
+    if (dev < 0 || dev >= MAX_DEVICES) return 0;
+    std::lock_guard<std::mutex> g(mu);
+    if (pairs[dev] == 0) {
+        if (cudaFuncSetAttribute(qkv_prologue_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(PCfg<DH>::SMEM_BYTES + 1024)) != cudaSuccess)
+            return 0;
+        cudaLaunchConfig_t cfg;
+        cudaLaunchAttribute attr[1];
+        pair_config<DH>(cfg, attr, 1, nullptr);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, qkv_prologue_kernel<DH>, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            return 0;
         }
+        pairs[dev] = n;
     }
-    qkv_prologue_kernel<DH><<<static_cast<unsigned>(grid), NTHREADS, smem, s>>>(prm);
+    return pairs[dev];
+}
+
+template <int DH>
+static int launch_kernel(const Params &prm, long long n_tiles, cudaStream_t s)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
+    const int fit = resident_pairs<DH>(dev);
+    if (fit < 1) return ATTN_JVP_ERR_LAUNCH;
+    const unsigned pairs = static_cast<unsigned>(n_tiles < fit ? n_tiles : fit);
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    pair_config<DH>(cfg, attr, pairs, s);
+    if (cudaLaunchKernelEx(&cfg, qkv_prologue_kernel<DH>, prm) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     return cudaGetLastError() == cudaSuccess ? ATTN_JVP_OK : ATTN_JVP_ERR_LAUNCH;
 }
 
@@ -393,7 +458,7 @@ int qkv_rmsnorm_jvp(const void *x, const void *x_dot, const void *w_qkv, const f
     if (d != 64 && d != 128) return ATTN_JVP_ERR_HEADDIM;
     const long long T = static_cast<long long>(B) * L;
     if (T >= (1ll << 31) || 3ll * H * d >= (1ll << 31)) return ATTN_JVP_ERR_SHAPE;
-    const long long n_tiles = ((T + BM - 1) / BM) * 3ll * H;
+    const long long n_tiles = ((T + 2 * BM - 1) / (2 * BM)) * 3ll * H;  // 256-token blocks x heads
     if (n_tiles > INT_MAX) return ATTN_JVP_ERR_SHAPE;
     const void *a16[9] = {x, x_dot, w_qkv, q, k, v, q_dot, k_dot, v_dot};
     for (const void *p : a16)
@@ -415,7 +480,7 @@ int qkv_rmsnorm_jvp(const void *x, const void *x_dot, const void *w_qkv, const f
     Params prm;
     std::memset(&prm, 0, sizeof prm);
     if (!make_map(&prm.tm_x, x, T, D, BM) || !make_map(&prm.tm_xd, x_dot, T, D, BM) ||
-        !make_map(&prm.tm_w, w_qkv, 3ll * H * d, D, d))
+        !make_map(&prm.tm_w, w_qkv, 3ll * H * d, D, d / 2))
         return ATTN_JVP_ERR_LAUNCH;
     prm.gamma_q = gamma_q;
     prm.gamma_k = gamma_k;
@@ -424,17 +489,12 @@ int qkv_rmsnorm_jvp(const void *x, const void *x_dot, const void *w_qkv, const f
     prm.L = L;
     prm.H = H;
     prm.D = D;
-    prm.tiles_m = static_cast<int>((T + BM - 1) / BM);
+    prm.tiles_m = static_cast<int>((T + 2 * BM - 1) / (2 * BM));
     prm.eps = eps;
     prm.timeout_ns = TIMEOUT_NS;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // persistent: one CTA per SM (or per tile, if there are fewer)
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
-        return ATTN_JVP_ERR_LAUNCH;
-    const long long grid = n_tiles < sms ? n_tiles : sms;
-    return d == 128 ? launch_kernel<128>(prm, grid, s) : launch_kernel<64>(prm, grid, s);
+    // persistent: as many CTA pairs as fit at once (or one per tile, if there are fewer)
+    return d == 128 ? launch_kernel<128>(prm, n_tiles, s) : launch_kernel<64>(prm, n_tiles, s);
 }
 
 int qkv_prologue_check(void *stream, int *site)
