@@ -197,6 +197,59 @@ def aggregate(local_ms: float, local_flops: float, group_active: bool, device=No
     return float(t.item()), float(f.item())
 
 
+E2E_NOTE = ("pipelined stream: every step copies its inputs host->device (pinned) and its "
+            "outputs device->host; two device buffer sets and three CUDA streams let step i+1's "
+            "input copies and step i-1's output copies overlap step i")
+
+
+def stream_e2e(dev, host_ins, out_like, call, steps, group):
+    """End-to-end time (ms) of a streaming loop through the public API.
+
+    Every step copies its inputs from pinned host memory to the device, runs
+    `call(dev_inputs, dev_outputs, stream)` and copies its outputs back to
+    pinned host memory.  Two device buffer sets and three streams (input
+    copies, compute, output copies) let the next step's inputs and the
+    previous step's outputs cross PCIe, in both directions at once, while a
+    step computes, as a user streaming batches would.  The timed region runs
+    from the first input copy to the last output copy."""
+    import torch
+    import torch.distributed as dist
+    slots_in = [[torch.empty(h.shape, dtype=h.dtype, device=dev) for h in host_ins] for _ in range(2)]
+    slots_out = [[torch.empty_like(o) for o in out_like] for _ in range(2)]
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in out_like]
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    torch.cuda.synchronize(dev)
+    if group:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for i in range(steps):
+        k = i % 2
+        if i >= 2:
+            s_in.wait_event(ev_comp[k])  # step i-2's kernel has read these inputs
+        with torch.cuda.stream(s_in):
+            for dst, src in zip(slots_in[k], host_ins):
+                dst.copy_(src, non_blocking=True)
+        ev_in[k].record(s_in)
+        s_comp.wait_event(ev_in[k])
+        if i >= 2:
+            s_comp.wait_event(ev_out[k])  # step i-2's outputs have left the device
+        call(slots_in[k], slots_out[k], s_comp)
+        ev_comp[k].record(s_comp)
+        s_out.wait_event(ev_comp[k])
+        with torch.cuda.stream(s_out):
+            for dst, src in zip(host_out, slots_out[k]):
+                dst.copy_(src, non_blocking=True)
+        ev_out[k].record(s_out)
+    e1.record(s_out)
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1)
+
+
 # ----------------------------------------------------------------- CPU oracle
 
 def time_oracle(w, seconds: float, seed: int = 123):
@@ -376,26 +429,13 @@ def run_ours(args):
 
     # end to end: pinned host inputs -> device, kernel, outputs -> pinned host
     e2e_steps = args.e2e_steps or min(args.steps, 100)
-    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    hod = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
-    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-    torch.cuda.synchronize(dev)
-    if group:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(e2e_steps):
-            for dst, src in zip(ins, host):
-                dst.copy_(src, non_blocking=True)
-            step()
-            ho.copy_(o, non_blocking=True)
-            hod.copy_(od, non_blocking=True)
-            hl.copy_(lse, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms, e2e_flops = aggregate(e0.elapsed_time(e1), flops_step * e2e_steps, group, dev)
+
+    def e2e_call(di, do, st):
+        ci = di[:4] + [None, None] if zkv else di
+        A.attn_jvp_fwd(*ci, scale=w.scale, kv_len=kv, out=tuple(do), stream=st)
+
+    e2e_local = stream_e2e(dev, host, (o, od, lse), e2e_call, e2e_steps, group)
+    e2e_ms, e2e_flops = aggregate(e2e_local, flops_step * e2e_steps, group, dev)
     e2e_value = e2e_flops / (e2e_ms * 1e-3) / 1e12
     h2d = in_bytes
     d2h = (o.numel() + od.numel()) * 2 + lse.numel() * 4
@@ -424,7 +464,7 @@ def run_ours(args):
                      "flops_per_launch": w.flops_performed(),
                      "kernel": f"attn_jvp_fwd_kernel<{d}>"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps, "how": E2E_NOTE},
         "clocks": clocks,
     }
     if w.kv_len is not None:
@@ -519,22 +559,12 @@ def run_loss(args):
     value = total_bytes / (max_ms * 1e-3) / 1e9
 
     e2e_steps = args.e2e_steps or min(args.steps, 100)
-    hl = torch.empty(B, dtype=torch.float32, pin_memory=True)
-    hg = torch.empty(grad.shape, dtype=grad.dtype, pin_memory=True)
-    torch.cuda.synchronize(dev)
-    if group:
-        dist.barrier()
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(e2e_steps):
-            for dst, src in zip(ins, host):
-                dst.copy_(src, non_blocking=True)
-            step()
-            hl.copy_(loss, non_blocking=True)
-            hg.copy_(grad, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms, e2e_bytes = aggregate(e0.elapsed_time(e1), bytes_step * e2e_steps, group, dev)
+
+    def e2e_call(di, do, st):
+        A.scm_tangent_loss(*di, out=tuple(do), stream=st)
+
+    e2e_local = stream_e2e(dev, host, (loss, grad), e2e_call, e2e_steps, group)
+    e2e_ms, e2e_bytes = aggregate(e2e_local, bytes_step * e2e_steps, group, dev)
 
     _, _, hbm, peak_src = load_peaks()
     achieved = bytes_step / (local_ms / args.steps * 1e-3) / 1e9
@@ -553,7 +583,7 @@ def run_loss(args):
                      "kernel": "scm_loss_kernel<1>"},
         "e2e": {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": 3 * B * N * 2, "d2h_bytes_per_step": B * N * 2 + 4 * B,
-                "steps": e2e_steps},
+                "steps": e2e_steps, "how": E2E_NOTE},
         "clocks": clocks,
     }
     if rank == 0 and not group and not args.no_cpu_baseline:
@@ -646,19 +676,12 @@ def run_qkv(args):
     value = total / (max_ms * 1e-3) / 1e12
 
     e2e_steps = args.e2e_steps or min(args.steps, 100)
-    hout = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(e2e_steps):
-            for dst, src in zip((x, xd, w), host):
-                dst.copy_(src, non_blocking=True)
-            step()
-            for h, o in zip(hout, outs):
-                h.copy_(o, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms, e2e_fl = aggregate(e0.elapsed_time(e1), flops_step * e2e_steps, group, dev)
+
+    def e2e_call(di, do, st):
+        A.qkv_rmsnorm_jvp(di[0], di[1], di[2], gq, gk, B, L, H, out=tuple(do), stream=st)
+
+    e2e_local = stream_e2e(dev, host, outs, e2e_call, e2e_steps, group)
+    e2e_ms, e2e_fl = aggregate(e2e_local, flops_step * e2e_steps, group, dev)
 
     burst_tf, sustained_tf, _, peak_src = load_peaks()
     if sustained_tf is not None and local_ms >= SUSTAINED_MS:
@@ -681,7 +704,8 @@ def run_qkv(args):
                      "traffic": measured_traffic("qkv_t2i", QKV_SOURCES), "flops_per_launch": flops_step,
                      "kernel": "qkv_prologue_kernel<128>"},
         "e2e": {"value": e2e_fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": in_bytes,
-                "d2h_bytes_per_step": sum(o.numel() * 2 for o in outs), "steps": e2e_steps},
+                "d2h_bytes_per_step": sum(o.numel() * 2 for o in outs), "steps": e2e_steps,
+                "how": E2E_NOTE},
         "clocks": clocks,
     }
     if rank == 0:
