@@ -51,21 +51,26 @@ def test_kv_len_and_nan_padding(d):
     compare(gpu_rows(*run_gpu(w)), oracle_ref(w), f"kv_len d{d}")
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("scale", [-0.3, 0.0, 2.0])
-def test_scale_values(scale):
-    w = W.make_custom(1, 3, 150, 300, 128, seed=9)
-    compare(gpu_rows(*run_gpu(w, scale=scale)), oracle_ref(w, scale=scale), f"scale {scale}")
+def test_scale_values(scale, d):
+    """A negative scale turns the row max into a row min; scale 0 makes P
+    uniform."""
+    w = W.make_custom(1, 3, 150, 300, d, seed=9)
+    compare(gpu_rows(*run_gpu(w, scale=scale)), oracle_ref(w, scale=scale), f"scale {scale} d{d}")
 
 
-def test_large_tangent_mean():
+@pytest.mark.parametrize("d", [64, 128])
+def test_large_tangent_mean(d):
     """Tangent logits with a large common row mean (K' = K + 50): the
-    centring constant keeps O' accurate."""
-    w = W.make_custom(1, 2, 256, 512, 128, seed=10)
+    centring constant keeps O' accurate (at d = 64 each softmax warpgroup
+    has its own, merged in the epilogue)."""
+    w = W.make_custom(1, 2, 256, 512, d, seed=10)
     kd = W.bf16_bits_to_f32(w.k_dot) + 50.0 * W.bf16_bits_to_f32(w.k)
     w.k_dot = W.bf16_round_bits(kd)
     qd = W.bf16_bits_to_f32(w.q_dot) + 20.0
     w.q_dot = W.bf16_round_bits(qd)
-    compare(gpu_rows(*run_gpu(w)), oracle_ref(w), "large tangent mean")
+    compare(gpu_rows(*run_gpu(w)), oracle_ref(w), f"large tangent mean d{d}")
 
 
 def test_deterministic_and_streams():
@@ -108,3 +113,25 @@ def test_persistent_tile_walk(d):
         for b in range(B):
             t[b, :, int(kv[b]):] = nan_bits
     compare(gpu_rows(*run_gpu(w)), oracle_ref(w), f"tile walk d{d}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_all_keys_masked(d):
+    """kv_len = 0 for every batch: no CTA has a key tile, so the loads, the
+    MMAs and the softmax loops all skip every query tile; O = O' = 0 and
+    lse = -inf everywhere."""
+    B, H, Lq, Lk = 3, 2, 200, 100
+    kv = np.zeros(B, np.int32)
+    w = W.make_custom(B, H, Lq, Lk, d, seed=14, kv_len=kv)
+    o, od, lse = run_gpu(w)
+    assert not torch.any(o.float() != 0) and not torch.any(od.float() != 0)
+    assert bool(torch.all(torch.isneginf(lse)))
+    compare(gpu_rows(o, od, lse), oracle_ref(w), f"all masked d{d}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_many_one_row_query_tiles(d):
+    """300 query tiles of 3 rows each (Lq = 3, 150 heads per batch): every
+    CTA walks two or three nearly empty query tiles."""
+    w = W.make_custom(2, 150, 3, 700, d, seed=15)
+    compare(gpu_rows(*run_gpu(w)), oracle_ref(w), f"one-row tiles d{d}")
