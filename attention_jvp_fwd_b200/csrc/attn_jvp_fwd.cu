@@ -918,6 +918,62 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
 #pragma unroll
                     for (int i = 0; i < 32; ++i) x[i] = (i < valid) ? x[i] : 0.f;
                 }
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+                if (j >= 1) {
+                    // PV of the previous key tile must be done before O may be
+                    // rescaled; every warp observes every phase of o_done in
+                    // order (phase gk needs this warp's P of key tile gk).
+                    if (!__all_sync(0xffffffffu, wait_bar_fast(&o_done[0], (gk - 1) & 1, wc, SITE_O_DONE))) {
+                        err = true;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                if (__any_sync(0xffffffffu, rescale)) {
+                    const uint32_t tacc = tbase + lane_off + (g == 0 ? C::T_O(0) : C::T_OD(0));
+#pragma unroll 1
+                    for (int c = 0; c < D; c += 32) {
+                        uint32_t tt[32];
+                        tmem_ld32(tacc + c, tt);
+                        tmem_ld_wait(tt);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) tt[i] = f2u(u2f(tt[i]) * alpha);
+                        tmem_st32(tacc + c, tt);
+                    }
+                }
+                if (tail && !(ZKV && g == 1)) {  // (no V' tile with V' = 0)
+                    // Zero the V (g = 0) / V' (g = 1) rows of padded keys so
+                    // their bits (NaN included) cannot reach the PV products.
+                    // Each warp zeroes its share and fences before it signals P.
+                    const int s = gk % C::NV;
+                    if (!__all_sync(0xffffffffu, wait_bar(&v_full[s], (gk / C::NV) & 1, wc, SITE_V_TAIL))) {
+                        err = true;
+                        if (j == 0) bar_and(BAR_SOFT, NSOFT, false);  // the others wait there at key tile 0
+                        break;
+                    }
+                    uint8_t *vst = smem + C::OFF_V + s * C::VST_BYTES + g * (C::NKB * BN * 128);
+                    const int nrow = BN - vt;
+                    const int per_blk = nrow * 8;
+                    const int chunks = C::NKB * per_blk;
+                    for (int idx = gt; idx < chunks; idx += 128) {
+                        const int blk = idx / per_blk;
+                        const int rem = idx - blk * per_blk;
+                        const int row = vt + (rem >> 3);
+                        *reinterpret_cast<uint4 *>(vst + blk * (BN * 128) + row * 128 + (rem & 7) * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                }
+                // P over the first 16 columns of this half of S'_raw (read above)
+                tmem_st16(tS + BN + c0, pk);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[bsel]);
+                // l, S'_raw and (first tile) the centring constant are needed
+                // only for P (sS' - c), so they come after P is on its way
                 {
                     uint64_t s0 = f2_pack(x[0], x[1]), s1 = f2_pack(x[2], x[3]);
 #pragma unroll
@@ -953,59 +1009,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                     if (g == 1) cctr = xch[512 + r];
                 }
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-                if (j >= 1) {
-                    // PV of the previous key tile must be done before O may be
-                    // rescaled; every warp observes every phase of o_done in
-                    // order (phase gk needs this warp's P of key tile gk).
-                    if (!__all_sync(0xffffffffu, wait_bar_fast(&o_done[0], (gk - 1) & 1, wc, SITE_O_DONE))) {
-                        err = true;
-                        break;
-                    }
-                    tc_fence_after();
-                }
-                if (__any_sync(0xffffffffu, rescale)) {
-                    const uint32_t tacc = tbase + lane_off + (g == 0 ? C::T_O(0) : C::T_OD(0));
-#pragma unroll 1
-                    for (int c = 0; c < D; c += 32) {
-                        uint32_t tt[32];
-                        tmem_ld32(tacc + c, tt);
-                        tmem_ld_wait(tt);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) tt[i] = f2u(u2f(tt[i]) * alpha);
-                        tmem_st32(tacc + c, tt);
-                    }
-                }
-                if (tail && !(ZKV && g == 1)) {  // (no V' tile with V' = 0)
-                    // Zero the V (g = 0) / V' (g = 1) rows of padded keys so
-                    // their bits (NaN included) cannot reach the PV products.
-                    // Each warp zeroes its share and fences before it signals P.
-                    const int s = gk % C::NV;
-                    if (!__all_sync(0xffffffffu, wait_bar(&v_full[s], (gk / C::NV) & 1, wc, SITE_V_TAIL))) {
-                        err = true;
-                        break;
-                    }
-                    uint8_t *vst = smem + C::OFF_V + s * C::VST_BYTES + g * (C::NKB * BN * 128);
-                    const int nrow = BN - vt;
-                    const int per_blk = nrow * 8;
-                    const int chunks = C::NKB * per_blk;
-                    for (int idx = gt; idx < chunks; idx += 128) {
-                        const int blk = idx / per_blk;
-                        const int rem = idx - blk * per_blk;
-                        const int row = vt + (rem >> 3);
-                        *reinterpret_cast<uint4 *>(vst + blk * (BN * 128) + row * 128 + (rem & 7) * 16) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                }
-                // P over the first 16 columns of this half of S'_raw (read above)
-                tmem_st16(tS + BN + c0, pk);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[bsel]);
                 // ---- bf16 P (s S' - c) while the tensor core multiplies P
                 uint32_t pdk[16];
                 {
