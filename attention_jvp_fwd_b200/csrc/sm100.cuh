@@ -78,21 +78,8 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Same probes with cluster-scope acquire, for barriers that the peer CTA of a
-// pair arrives on.
-__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
+// mbar_try_wait with cluster-scope acquire, for barriers that the other CTA
+// of a pair arrives on (or that a pair commit signals).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
@@ -426,18 +413,6 @@ __device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
-__device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // Arrive once on the mbarrier at this shared-memory offset in every CTA of
 // `cta_mask` when the pair MMAs issued so far are done.
 __device__ __forceinline__ void mma_commit_pair_mc(uint64_t *bar, uint16_t cta_mask)
@@ -552,13 +527,5 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return r;
 }
 
-// fp32 -> bf16 on the integer pipe: add half a bf16 ulp to the bit pattern
-// (round to nearest, ties away from zero).  The upper 16 bits of the result
-// are the bf16 value; (r & 0xFFFF0000) is that value as fp32.  For the finite
-// MMA operands P and P (sS' - c).
-__device__ __forceinline__ uint32_t round_bf16_bits(float x)
-{
-    return __float_as_uint(x) + 0x8000u;
-}
 
 }  // namespace ajvp
