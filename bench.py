@@ -612,6 +612,97 @@ QKV_METRIC = "QKV projection + RMSNorm forward-and-tangent TFLOP/s (2 GEMMs, 2*2
 QKV_SHAPE = dict(B=2, L=4096, H=16, D=2048, d=128)
 
 
+def qkv_inputs(seed: int):
+    """Seeded bf16 bits of x, x' [T, D] (N(0, 1)) and W [3Hd, D] (N(0, 1/D))."""
+    from attention_jvp_fwd_b200.workloads import bf16_round_bits
+    B, L, H, D, d = (QKV_SHAPE[k] for k in ("B", "L", "H", "D", "d"))
+    T = B * L
+    r = np.random.default_rng([seed, 13])
+    return [bf16_round_bits(r.standard_normal((T, D), dtype=np.float32)),
+            bf16_round_bits(r.standard_normal((T, D), dtype=np.float32)),
+            bf16_round_bits((r.standard_normal((3 * H * d, D)) / np.sqrt(D)).astype(np.float32))]
+
+
+def time_qkv_oracle(bits, seconds: float):
+    """The fp64 prologue oracle on the first `n` tokens per call (all heads),
+    n sized for about `seconds`; returns (TFLOP/s, tokens per call, calls, s)."""
+    from oracle import qkv_prologue
+    H, D, d = QKV_SHAPE["H"], QKV_SHAPE["D"], QKV_SHAPE["d"]
+    x, xd, w = bits
+    one = np.ones(d)
+    n, calls, dt = 16, 0, 0.0
+    while True:
+        t0 = time.perf_counter()
+        qkv_prologue.qkv_rmsnorm_jvp(x[:n], xd[:n], w, one, one, 1, n, H, d)
+        dt1 = time.perf_counter() - t0
+        if dt1 > seconds / 8 or n >= x.shape[0]:
+            break
+        n = min(x.shape[0], n * 2)
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds or calls == 0:
+        qkv_prologue.qkv_rmsnorm_jvp(x[:n], xd[:n], w, one, one, 1, n, H, d)
+        calls += 1
+    dt = time.perf_counter() - t0
+    flops = 2.0 * 2 * n * D * 3 * H * d * calls
+    return flops / dt / 1e12, n, calls, dt
+
+
+def run_reference_qkv(args):
+    """``--impl reference --workload qkv_t2i``: the fp64 oracle of the prologue
+    on the host cores, on bounded token samples of the same layer."""
+    _, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    bits = qkv_inputs(args.seed)
+    per_step = max(1.0, min(20.0, 120.0 / (args.steps + args.warmup)))
+    time_qkv_oracle(bits, per_step * args.warmup / max(1, args.steps))  # warm-up
+    v, n, calls, dt = time_qkv_oracle(bits, per_step * args.steps)
+    sample = (f"first {n} tokens of the layer (all {3 * QKV_SHAPE['H']} head tiles) per call, "
+              f"{calls} calls, {dt:.1f} s; numpy fp64")
+    line = {"metric": QKV_METRIC, "value": v, "unit": "TFLOP/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "qkv_t2i", **QKV_SHAPE, "seed": args.seed},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference_loss(args):
+    """``--impl reference --workload scm_loss``: the fp64 oracle of the loss on
+    the host cores, one sample per call."""
+    _, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    from oracle import scm_loss
+    bits = loss_inputs(args.seed)
+    B = LOSS_SHAPE[0]
+    N = int(np.prod(LOSS_SHAPE[1:]))
+    budget = max(1.0, min(20.0, 120.0 / (args.steps + args.warmup)))
+    for i in range(args.warmup):
+        scm_loss.scm_tangent_loss(*[b[i % B:i % B + 1].reshape(1, -1) for b in bits])
+    n = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget * args.steps or n == 0:
+        scm_loss.scm_tangent_loss(*[b[n % B:n % B + 1].reshape(1, -1) for b in bits])
+        n += 1
+    dt = time.perf_counter() - t0
+    v = n * (4.0 * N * 2 + 4) / dt / 1e9
+    line = {"metric": LOSS_METRIC, "value": v, "unit": "GB/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "scm_loss", "shape": list(LOSS_SHAPE), "c": 0.1, "seed": args.seed},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{n} single-sample calls ({N} elements each), {dt:.1f} s; numpy fp64"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_qkv(args):
     """``--workload qkv_t2i``: the prologue kernel (a tensor-core GEMM pair with
     an RMSNorm-JVP epilogue) on a T2I-sized layer."""
@@ -630,14 +721,10 @@ def run_qkv(args):
     if group:
         dist.barrier()
     import attention_jvp_fwd_b200 as A
-    from attention_jvp_fwd_b200.workloads import bf16_round_bits
 
     B, L, H, D, d = (QKV_SHAPE[k] for k in ("B", "L", "H", "D", "d"))
     T = B * L
-    r = np.random.default_rng([args.seed + rank, 13])
-    bits = [bf16_round_bits(r.standard_normal((T, D), dtype=np.float32)),
-            bf16_round_bits(r.standard_normal((T, D), dtype=np.float32)),
-            bf16_round_bits((r.standard_normal((3 * H * d, D)) / np.sqrt(D)).astype(np.float32))]
+    bits = qkv_inputs(args.seed + rank)
     host = [torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).pin_memory() for b in bits]
     x, xd, w = (h.to(dev, non_blocking=True) for h in host)
     gq = torch.ones(d, dtype=torch.float32, device=dev)
@@ -708,6 +795,11 @@ def run_qkv(args):
                 "how": E2E_NOTE},
         "clocks": clocks,
     }
+    if rank == 0 and not group and not args.no_cpu_baseline:
+        v, n, calls, dt = time_qkv_oracle(bits, min(args.cpu_seconds, 10.0))
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                                "sample": f"first {n} tokens (all head tiles) per call, {calls} calls, "
+                                          f"{dt:.1f} s; numpy fp64"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if group:
@@ -719,17 +811,9 @@ def run_qkv(args):
 def main(argv=None):
     args = parse_args(argv)
     if args.workload == "qkv_t2i":
-        if args.impl == "reference":
-            print(json.dumps({"impl": "reference", "unavailable":
-                              "the prologue leg has no reference arm; run the attention workloads"}))
-            return 0
-        return run_qkv(args)
+        return run_reference_qkv(args) if args.impl == "reference" else run_qkv(args)
     if args.workload == "scm_loss":
-        if args.impl == "reference":
-            print(json.dumps({"impl": "reference", "unavailable":
-                              "the sCM loss leg has no reference arm; run the attention workloads"}))
-            return 0
-        return run_loss(args)
+        return run_reference_loss(args) if args.impl == "reference" else run_loss(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
