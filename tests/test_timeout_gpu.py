@@ -13,12 +13,17 @@ from gpu_util import compare, gpu_rows, oracle_ref, to_dev
 pytestmark = pytest.mark.gpu
 
 
-def test_starved_wait_reports_timeout_and_recovers():
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B,H,Lq", [(1, 2, 256), (2, 100, 300)])
+def test_starved_wait_reports_timeout_and_recovers(d, B, H, Lq):
+    """Both softmax splits (d = 64 by key tiles, d = 128 by columns); the
+    second shape has 600 query tiles, so every persistent CTA has more tiles
+    queued when the wait gives up."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from attention_jvp_fwd_b200.build import build
     build()
-    w = W.make_custom(1, 2, 256, 1024, 128, seed=3)
+    w = W.make_custom(B, H, Lq, 1024, d, seed=3)
     ins = [to_dev(x) for x in w.inputs()]
     assert A.attn_jvp_check()[0] == A.ATTN_JVP_OK
     A.attn_jvp_fwd(*ins, scale=w.scale, _debug_timeout_ns=2_000_000,
@@ -29,4 +34,4 @@ def test_starved_wait_reports_timeout_and_recovers():
     assert A.attn_jvp_check()[0] == A.ATTN_JVP_OK
     o, od, lse = A.attn_jvp_fwd(*ins, scale=w.scale)
     assert A.attn_jvp_check()[0] == A.ATTN_JVP_OK
-    compare(gpu_rows(o, od, lse), oracle_ref(w), "after timeout")
+    compare(gpu_rows(o, od, lse), oracle_ref(w), f"after timeout d{d} B{B} H{H}")
