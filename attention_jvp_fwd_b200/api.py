@@ -25,9 +25,10 @@ ATTN_JVP_ERR_TIMEOUT = -6
 ATTN_JVP_ERR_VALUE = -7
 ATTN_JVP_DEBUG_STARVE_Q = 1
 
-EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_ex", "attn_jvp_fwd_debug", "attn_jvp_check",
-            "attn_jvp_status_string", "attn_jvp_version", "scm_tangent_loss", "qkv_rmsnorm_jvp",
-            "qkv_prologue_check")
+EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_ex", "attn_jvp_fwd_debug", "attn_jvp_fwd_trace",
+            "attn_jvp_check", "attn_jvp_status_string", "attn_jvp_version", "scm_tangent_loss",
+            "qkv_rmsnorm_jvp", "qkv_prologue_check")
+TRACE_EVENTS = 11  # stamps per key tile of attn_jvp_fwd_trace
 
 _lock = threading.Lock()
 _lib = None
@@ -68,6 +69,8 @@ def load_library():
             lib.attn_jvp_fwd_debug.restype = i32
             lib.attn_jvp_fwd_debug.argtypes = [vp] * 9 + [i32] * 5 + [f32, vp, vp,
                                                                      ctypes.c_uint64, i32]
+            lib.attn_jvp_fwd_trace.restype = i32
+            lib.attn_jvp_fwd_trace.argtypes = [vp] * 9 + [i32] * 5 + [f32, vp, vp, vp, i32, i32]
             lib.attn_jvp_check.restype = i32
             lib.attn_jvp_check.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
             lib.attn_jvp_status_string.restype = ctypes.c_char_p
@@ -178,6 +181,42 @@ def attn_jvp_fwd(q, k, v, q_dot, k_dot, v_dot, scale: float | None = None, kv_le
     if rc != ATTN_JVP_OK:
         raise AttnJvpError(rc, "attn_jvp_fwd")
     return (o, od, lse, ld) if lse_dot else (o, od, lse)
+
+
+def attn_jvp_fwd_trace(q, k, v, q_dot, k_dot, v_dot, scale: float | None = None, kv_len=None,
+                       tiles: int = 64, ctas: int | None = None, stream=None):
+    """attn_jvp_fwd in the trace build: returns (o, o_dot, lse, trace), where
+    trace is int64 [ctas, tiles, TRACE_EVENTS] of SM clock stamps of each
+    CTA's first ``tiles`` key tiles (0 where no stamp was taken); ``ctas``
+    defaults to the SM count.  The outputs equal attn_jvp_fwd's bit for bit.
+    See attention_jvp_fwd_b200.trace for the event list and a summary."""
+    B, H, Lq, Lk, d = _check_inputs(q, k, v, q_dot, k_dot, v_dot)
+    if k_dot is None:
+        raise ValueError("the trace build takes all six inputs")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    kv_ptr = None
+    if kv_len is not None:
+        if (not isinstance(kv_len, torch.Tensor) or kv_len.dtype != torch.int32
+                or kv_len.device != q.device or tuple(kv_len.shape) != (B,)
+                or not kv_len.is_contiguous()):
+            raise ValueError("kv_len must be a contiguous int32 [B] tensor on q's device")
+        kv_ptr = kv_len.data_ptr()
+    if ctas is None:
+        ctas = torch.cuda.get_device_properties(q.device).multi_processor_count
+    o = torch.empty_like(q)
+    od = torch.empty_like(q)
+    lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    trace = torch.zeros((ctas, tiles, TRACE_EVENTS), dtype=torch.int64, device=q.device)
+    lib = load_library()
+    ptrs = [t.data_ptr() for t in (q, k, v, q_dot, k_dot, v_dot, o, od, lse)]
+    with torch.cuda.device(q.device):
+        rc = lib.attn_jvp_fwd_trace(*ptrs, B, H, Lq, Lk, d, float(scale), kv_ptr,
+                                    _stream_handle(q.device, stream), trace.data_ptr(), int(tiles),
+                                    int(ctas))
+    if rc != ATTN_JVP_OK:
+        raise AttnJvpError(rc, "attn_jvp_fwd_trace")
+    return o, od, lse, trace
 
 
 def attn_jvp_check(stream=None, device=None) -> tuple[int, int]:

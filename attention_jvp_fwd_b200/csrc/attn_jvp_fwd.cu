@@ -127,6 +127,10 @@ struct Cfg {
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, 2 * BN, false);
     static constexpr uint32_t IDESC_SD = idesc_bf16_f32(BM, BN, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
+    // P [V | V'] into [O | O'_acc] as one N = 2d MMA: the V stage holds V's
+    // and then V''s 64-column blocks at one stride, and O'_acc follows O in TMEM
+    static constexpr uint32_t IDESC_PVV = idesc_bf16_f32(BM, 2 * D, true);
+    static_assert(2 * D <= 256, "one MMA covers at most 256 columns");
     static constexpr int P_ARRIVALS = ALT ? 4 : 8;  // one per softmax warp that writes the tile
     static_assert(T_S + 4 * BN <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -144,6 +148,23 @@ struct Params {
     float sl2;    // s * log2(e)
     uint64_t timeout_ns;
     int flags;
+    // trace build only: clock64 stamps [trace_ctas][trace_tiles][TRACE_EVENTS]
+    unsigned long long *trace;
+    int trace_tiles, trace_ctas;
+};
+
+// Events a trace build stamps for each of a CTA's key tiles (gg counts the
+// key tiles of all the CTA's query tiles), in SM clock cycles.
+enum : int {
+    EV_K_LOAD = 0,   // TMA warp: K/K' loads issued
+    EV_V_LOAD = 1,   // TMA warp: V/V' loads issued
+    EV_S_ISSUE = 2,  // MMA warp: S and S' MMAs issued
+    EV_PA_ISSUE = 3, // MMA warp: P V (and P V') MMAs issued
+    EV_PB_ISSUE = 4, // MMA warp: P (sS' - c) V MMAs issued
+    EV_SM_S = 5,     // softmax, first warp of warpgroup g: S seen   (+ 3g)
+    EV_SM_P = 6,     // softmax: bf16 P stored and signalled          (+ 3g)
+    EV_SM_PD = 7,    // softmax: bf16 P (sS' - c) stored and signalled (+ 3g)
+    TRACE_EVENTS = 11,
 };
 
 // One query tile: rows q0 .. q0 + 127 of head bh, against the nb valid keys
@@ -241,10 +262,17 @@ __device__ __forceinline__ float row_min64(const uint32_t (&a)[32], const uint32
 // way, so the key tiles of all its query tiles form one sequence gg = 0, 1,
 // ...: the K and V ring slots, the S/P TMEM buffer and the phases of the
 // per-key-tile barriers all follow gg.
-template <int D, bool ZKV>
+template <int D, bool ZKV, bool TRACE>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_constant__ Params p)
 {
     using C = Cfg<D>;
+    // trace build: stamp event `ev` of key tile gk (no code in the normal build)
+    auto stamp = [&](const int gk, const int ev) {
+        if constexpr (TRACE) {
+            if (gk < p.trace_tiles && static_cast<int>(blockIdx.x) < p.trace_ctas)
+                p.trace[(static_cast<size_t>(blockIdx.x) * p.trace_tiles + gk) * TRACE_EVENTS + ev] = clock64();
+        }
+    };
     extern __shared__ __align__(1024) uint8_t smem[];
     // The 128-byte swizzle atoms must start on 1024-byte boundaries.  The
     // dynamic window is 1024-aligned in practice; if it ever is not, record it
@@ -364,6 +392,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                                 tma_load_3d(dst + c * (2 * BN * 128) + BN * 128, &p.tm_kd, &k_full[s], c * 64,
                                             j * BN, t.bh, pol_kv);
                         }
+                        stamp(kc, EV_K_LOAD);
                         ++kc;
                     }
                     if (j >= 1) {
@@ -380,6 +409,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                                 tma_load_3d(dst + (C::NKB + c) * (BN * 128), &p.tm_vd, &v_full[s], c * 64,
                                             (j - 1) * BN, t.bh, pol_kv);
                         }
+                        stamp(vc, EV_V_LOAD);
                         ++vc;
                     }
                 }
@@ -454,18 +484,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const uint32_t tP = tbase + C::T_S + (gk & 1) * (2 * BN);
             const int ow = C::ALT ? (gk & 1) : 0;
             const uint64_t dv = sdesc_sw128(smem_addr(smem + C::OFF_V + s * C::VST_BYTES), LBO, 1024);
-            const uint64_t dvd = desc_add(dv, C::VHALF_BYTES);
-            (void)dvd;
+            static_assert(C::VHALF_BYTES == C::NKB * LBO, "V' blocks follow V's at the block stride");
 #pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)  // O += P V
-                mma_ts(tbase + C::T_O(ow), tP + C::t_pk(kk, false), desc_add(dv, kk * 2048), C::IDESC_PV,
-                       (!first || kk > 0) ? 1u : 0u);
-            if constexpr (!ZKV) {
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)  // O'_acc += P V'
-                    mma_ts(tbase + C::T_OD(ow), tP + C::t_pk(kk, false), desc_add(dvd, kk * 2048), C::IDESC_PV,
-                           (!first || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < BN / 16; ++kk)  // [O | O'_acc] += P [V | V']  (with V' = 0: O += P V)
+                mma_ts(tbase + C::T_O(ow), tP + C::t_pk(kk, false), desc_add(dv, kk * 2048),
+                       ZKV ? C::IDESC_PV : C::IDESC_PVV, (!first || kk > 0) ? 1u : 0u);
         };
         auto issue_pb = [&](const int gk, const bool first) {
             const int s = gk % C::NV;
@@ -497,6 +520,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             if (ok) ok = wait_u(&k_full[gg % C::NK], (gg / C::NK) & 1, SITE_K_FULL);
             if (!ok) break;
             issue_s(gg);
+            if (lane == 0) stamp(gg, EV_S_ISSUE);
             if (t.nT == 1) mma_commit(q_empty);
             for (int j = 0; j < t.nT; ++j) {
                 const int gk = gg + j;
@@ -504,6 +528,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     ok = wait_u(&k_full[(gk + 1) % C::NK], ((gk + 1) / C::NK) & 1, SITE_K_FULL);
                     if (!ok) break;
                     issue_s(gk + 1);
+                    if (lane == 0) stamp(gk + 1, EV_S_ISSUE);
                     if (j + 2 == t.nT) mma_commit(q_empty);  // that was the tile's last S
                 }
                 // V_j normally lands before P_j is written: wait for it first
@@ -512,9 +537,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 if (!ok) break;
                 const bool first = C::ALT ? j < 2 : j == 0;
                 issue_pa(gk, first);
+                if (lane == 0) stamp(gk, EV_PA_ISSUE);
                 ok = wait_u(&pd_full[gk & 1], (gk >> 1) & 1, SITE_P_FULL);
                 if (!ok) break;
                 issue_pb(gk, first);
+                if (lane == 0) stamp(gk, EV_PB_ISSUE);
             }
             gg += t.nT;
         }
@@ -534,6 +561,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         const int r = quad * 32 + lane;
         const int gt = tid - 64 - g * 128;  // thread index inside the warpgroup
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+        const bool tracer = TRACE && gt == 0;  // lane 0 of the warpgroup's first warp
         float *xch = reinterpret_cast<float *>(smem + C::OFF_XCH);
         const float sl2 = p.sl2;
         const float sc = p.scale;
@@ -569,6 +597,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         err = true;
                         break;
                     }
+                    if (tracer) stamp(gk, EV_SM_S + 3 * g);
                     tc_fence_after();
                     const int vt = nb - j * BN;  // valid keys in the tile
                     const bool tail = vt < BN;
@@ -685,6 +714,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&p_full[g]);
+                    if (tracer) stamp(gk, EV_SM_P + 3 * g);
                     // ---- bf16 P (s S' - c) while the tensor core multiplies P
                     tmem_ld_wait(rd);
                     if (nown == 0) {
@@ -741,6 +771,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pd_full[g]);
+                    if (tracer) stamp(gk, EV_SM_PD + 3 * g);
                     ++nown;
                     last = gk;
                 }
@@ -864,6 +895,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     if (j == 0) bar_and(BAR_SOFT, NSOFT, false);  // the others wait there at key tile 0
                     break;
                 }
+                if (tracer) stamp(gk, EV_SM_S + 3 * g);
                 tc_fence_after();
                 const int vt = nb - j * BN;  // valid keys in the tile
                 const int valid = vt - c0;   // valid columns of this half
@@ -972,6 +1004,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full[bsel]);
+                if (tracer) stamp(gk, EV_SM_P + 3 * g);
                 // l, S'_raw and (first tile) the centring constant are needed
                 // only for P (sS' - c), so they come after P is on its way
                 {
@@ -1041,6 +1074,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&pd_full[bsel]);
+                if (tracer) stamp(gk, EV_SM_PD + 3 * g);
             }
             bool ok;
             {
@@ -1147,7 +1181,7 @@ constexpr int MAX_DEVICES = 64;
 
 // Per device, once: the kernel's shared-memory opt-in and the SM count
 // (one persistent CTA per SM).
-template <int D, bool ZKV>
+template <int D, bool ZKV, bool TRACE>
 static int prepare_device(int dev, int *n_sm)
 {
     static std::mutex mu;
@@ -1156,7 +1190,7 @@ static int prepare_device(int dev, int *n_sm)
     if (dev < 0 || dev >= MAX_DEVICES) return ATTN_JVP_ERR_LAUNCH;
     std::lock_guard<std::mutex> g(mu);
     if (!done[dev]) {
-        if (cudaFuncSetAttribute(attn_jvp_fwd_kernel<D, ZKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(attn_jvp_fwd_kernel<D, ZKV, TRACE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(Cfg<D>::SMEM_BYTES)) != cudaSuccess)
             return ATTN_JVP_ERR_LAUNCH;
         if (cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms[dev] < 1)
@@ -1167,14 +1201,14 @@ static int prepare_device(int dev, int *n_sm)
     return ATTN_JVP_OK;
 }
 
-template <int D, bool ZKV>
+template <int D, bool ZKV, bool TRACE = false>
 static int launch_kernel(const Params &prm, cudaStream_t s)
 {
     int dev = 0, n_sm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
-    if (int rc = prepare_device<D, ZKV>(dev, &n_sm)) return rc;
+    if (int rc = prepare_device<D, ZKV, TRACE>(dev, &n_sm)) return rc;
     const int grid = prm.n_tiles < n_sm ? prm.n_tiles : n_sm;
-    attn_jvp_fwd_kernel<D, ZKV><<<grid, NTHREADS, Cfg<D>::SMEM_BYTES, s>>>(prm);
+    attn_jvp_fwd_kernel<D, ZKV, TRACE><<<grid, NTHREADS, Cfg<D>::SMEM_BYTES, s>>>(prm);
     return ATTN_JVP_OK;
 }
 
@@ -1185,14 +1219,18 @@ static bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb)
 }
 
 // allow_zero_kv: k_dot and v_dot may both be NULL (K' = V' = 0).
+// trace != NULL: the trace build, stamping [trace_ctas][trace_tiles][TRACE_EVENTS].
 static int launch(const void *q, const void *k, const void *v, const void *qd, const void *kd,
                   const void *vd, void *o, void *od, float *lse, float *lse_dot, int B, int H, int Lq,
                   int Lk, int d, float scale, const int32_t *kv_len, void *stream, uint64_t timeout_ns,
-                  int flags, bool allow_zero_kv)
+                  int flags, bool allow_zero_kv, unsigned long long *trace = nullptr, int trace_tiles = 0,
+                  int trace_ctas = 0)
 {
     const bool zkv = allow_zero_kv && !kd && !vd;
     if (!q || !k || !v || !qd || (!zkv && (!kd || !vd)) || !o || !od || !lse) return ATTN_JVP_ERR_NULL;
     if (flags & ~ATTN_JVP_DEBUG_STARVE_Q) return ATTN_JVP_ERR_VALUE;
+    if (trace && (trace_tiles < 1 || trace_ctas < 1 || (reinterpret_cast<uintptr_t>(trace) & 7)))
+        return trace_tiles < 1 || trace_ctas < 1 ? ATTN_JVP_ERR_VALUE : ATTN_JVP_ERR_ALIGN;
     if (B < 1 || H < 1 || Lq < 1 || Lk < 1) return ATTN_JVP_ERR_SHAPE;
     const long long BH = static_cast<long long>(B) * H;
     if (BH * Lq >= (1ll << 31) || BH * Lk >= (1ll << 31)) return ATTN_JVP_ERR_SHAPE;
@@ -1208,13 +1246,14 @@ static int launch(const void *q, const void *k, const void *v, const void *qd, c
     const size_t nl = static_cast<size_t>(BH) * Lq * 4;
     const void *ins[6] = {q, k, v, qd, kd, vd};
     const size_t insz[6] = {nq, nk, nk, nq, nk, nk};
-    const void *outs[4] = {o, od, lse, lse_dot};
-    const size_t outsz[4] = {nq, nq, nl, nl};
-    for (int i = 0; i < 4; ++i) {
+    const size_t ntr = trace ? static_cast<size_t>(trace_ctas) * trace_tiles * TRACE_EVENTS * 8 : 0;
+    const void *outs[5] = {o, od, lse, lse_dot, trace};
+    const size_t outsz[5] = {nq, nq, nl, nl, ntr};
+    for (int i = 0; i < 5; ++i) {
         if (!outs[i]) continue;
         for (int j = 0; j < 6; ++j)
             if (ins[j] && ranges_overlap(outs[i], outsz[i], ins[j], insz[j])) return ATTN_JVP_ERR_VALUE;
-        for (int j = i + 1; j < 4; ++j)
+        for (int j = i + 1; j < 5; ++j)
             if (outs[j] && ranges_overlap(outs[i], outsz[i], outs[j], outsz[j])) return ATTN_JVP_ERR_VALUE;
     }
 
@@ -1241,10 +1280,14 @@ static int launch(const void *q, const void *k, const void *v, const void *qd, c
     prm.sl2 = scale * 1.4426950408889634f;
     prm.timeout_ns = timeout_ns ? timeout_ns : DEFAULT_TIMEOUT_NS;
     prm.flags = flags;
+    prm.trace = trace;
+    prm.trace_tiles = trace_tiles;
+    prm.trace_ctas = trace_ctas;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int rc;
-    if (zkv) rc = d == 64 ? launch_kernel<64, true>(prm, s) : launch_kernel<128, true>(prm, s);
+    if (trace) rc = d == 64 ? launch_kernel<64, false, true>(prm, s) : launch_kernel<128, false, true>(prm, s);
+    else if (zkv) rc = d == 64 ? launch_kernel<64, true>(prm, s) : launch_kernel<128, true>(prm, s);
     else rc = d == 64 ? launch_kernel<64, false>(prm, s) : launch_kernel<128, false>(prm, s);
     if (rc) return rc;
     if (cudaGetLastError() != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
@@ -1278,6 +1321,16 @@ int attn_jvp_fwd_debug(const void *q, const void *k, const void *v, const void *
 {
     return ajvp::launch(q, k, v, q_dot, k_dot, v_dot, o, o_dot, lse, nullptr, B, H, Lq, Lk, d, scale,
                         kv_len, stream, timeout_ns, flags, false);
+}
+
+int attn_jvp_fwd_trace(const void *q, const void *k, const void *v, const void *q_dot,
+                       const void *k_dot, const void *v_dot, void *o, void *o_dot, float *lse, int B,
+                       int H, int Lq, int Lk, int d, float scale, const int32_t *kv_len, void *stream,
+                       unsigned long long *trace, int trace_tiles, int trace_ctas)
+{
+    if (!trace) return ATTN_JVP_ERR_NULL;
+    return ajvp::launch(q, k, v, q_dot, k_dot, v_dot, o, o_dot, lse, nullptr, B, H, Lq, Lk, d, scale,
+                        kv_len, stream, 0, 0, false, trace, trace_tiles, trace_ctas);
 }
 
 int attn_jvp_check(void *stream, int *site)

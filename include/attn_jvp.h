@@ -126,6 +126,34 @@ int attn_jvp_check(void *stream, int *site);
 const char *attn_jvp_status_string(int status);
 
 /*
+ * attn_jvp_fwd_trace -- attn_jvp_fwd in the trace build: the same results,
+ * bit for bit, plus SM clock stamps (clock64) of the pipeline events of each
+ * key tile, for measuring where the time of a key tile goes.  No counterpart
+ * on the pages: it exists to profile the kernel.
+ *   trace        device buffer of uint64 [trace_ctas][trace_tiles][11], written
+ *                where a stamp is taken and left as it was elsewhere; 8-byte
+ *                aligned, not overlapping any other argument
+ *   trace_tiles  key tiles stamped per CTA (a CTA counts the key tiles of all
+ *                its query tiles in order), >= 1
+ *   trace_ctas   CTAs stamped (blockIdx < trace_ctas), >= 1; the launch has
+ *                min(query tiles, SM count) CTAs
+ * Events per key tile (cycles of the CTA's SM; compare within a CTA only):
+ *   0 K/K' loads issued, 1 V/V' loads issued, 2 S MMAs issued, 3 P V MMAs
+ *   issued, 4 P (sS' - c) V MMAs issued; then for softmax warpgroup g = 0, 1
+ *   (the warpgroup's first warp): 5 + 3g S seen, 6 + 3g P signalled,
+ *   7 + 3g P (sS' - c) signalled.  At d = 64 warpgroup g handles the key tiles
+ *   with index % 2 == g, so only its events are stamped for them.
+ * Returns what attn_jvp_fwd returns, or ATTN_JVP_ERR_NULL (trace NULL),
+ * _VALUE (trace_tiles or trace_ctas < 1, or overlap), _ALIGN.
+ */
+int attn_jvp_fwd_trace(const void *q, const void *k, const void *v,
+                       const void *q_dot, const void *k_dot, const void *v_dot,
+                       void *o, void *o_dot, float *lse,
+                       int B, int H, int Lq, int Lk, int d, float scale,
+                       const int32_t *kv_len, void *stream,
+                       unsigned long long *trace, int trace_tiles, int trace_ctas);
+
+/*
  * attn_jvp_fwd_debug -- test hook: attn_jvp_fwd with an explicit wait limit
  * and fault-injection flags, so a test can make a device-side wait run out
  * without hanging or faulting the GPU.
