@@ -13,14 +13,19 @@
 //     K' sit next to each other in shared memory, so Q [K ; K']^T is a single
 //     N = 128 MMA that writes S and Q K'^T side by side; Q' K^T then adds onto
 //     the second half.  Together this is the K = 2d product [Q | Q'][K' | K]^T;
-//   * two warpgroups run the online softmax in registers, thread = query row,
-//     each on one half of the tile's 64 keys: running max m (lazily
-//     rescaled), denominator l = sum p and a = sum p (s S'_raw - c).  They
-//     write P and P (s S'_raw - c) back into TMEM as bf16 over S'_raw;
-//   * O += P V and O'_acc += P V' + P(sS' - c) V are tcgen05 MMAs with A read
-//     from TMEM;
+//   * two warpgroups run the online softmax in registers, thread = query row:
+//     running max m (lazily rescaled), denominator l = sum p and
+//     a = sum p (s S'_raw - c).  At d = 128 each takes one half of every
+//     tile's 64 keys; at d = 64 each takes every other key tile, with its own
+//     m, l, a and accumulators, merged at the end.  They write P and
+//     P (s S'_raw - c) back into TMEM as bf16;
+//   * [O | O'_acc] += P [V | V'] (one N = 2d MMA chain) and O'_acc +=
+//     P(sS' - c) V are tcgen05 MMAs with A read from TMEM;
 //   * the epilogue forms O = O_acc / l and O' = (O'_acc - (a / l) O_acc) / l,
 //     while the first S MMAs and loads of the next query tile already run.
+//
+// A trace instantiation (TRACE) stamps clock64 at each key tile's pipeline
+// events into a caller buffer; it computes the same results.
 //
 // c is a per-row constant (the p-weighted mean of s S'_raw over the first 32
 // keys).  In exact arithmetic O' does not depend on it; it keeps the bf16
