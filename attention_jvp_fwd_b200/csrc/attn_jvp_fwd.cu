@@ -101,9 +101,9 @@ struct Cfg {
     static constexpr uint32_t OFF_K = 2 * Q_BYTES;
     static constexpr uint32_t OFF_V = OFF_K + NK * KST_BYTES;
     static constexpr uint32_t OFF_BAR = OFF_V + NV * VST_BYTES;
-    // q_full, q_empty, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV],
-    // s_full[2], p_full[2], pd_full[2], o_done[2], drain
-    static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 2 + 1;
+    // q_full, q_empty, k_full[NK], ks_done[NK], v_full[NV], vo_done[NV],
+    // p_full[2], pd_full[2], drain, and by tiles s_full[2], o_done[2]
+    static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 2 + 2 + 1 + (ALT ? 4 : 0);
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem slot, abort flag
     // Softmax exchange, floats.  By columns: per-warpgroup partial l, a
     // ([2][2][128]) and the centring constant hand-off ([128]).  By tiles:
@@ -295,16 +295,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
     uint64_t *q_full = bars;
     uint64_t *q_empty = q_full + 1;  // the last S MMA of a query tile has read Q, Q'
     uint64_t *k_full = q_empty + 1;
-    uint64_t *k_empty = k_full + C::NK;
-    uint64_t *v_full = k_empty + C::NK;
-    uint64_t *v_empty = v_full + C::NV;
-    uint64_t *s_full = v_empty + C::NV;
-    uint64_t *p_full = s_full + 2;   // [2] bf16 P written
-    uint64_t *pd_full = p_full + 2;  // [2] bf16 P (sS' - c) written
-    // [2] the PV MMAs of a key tile are done: by columns o_done[0] has one
-    // phase per key tile; by tiles o_done[g] one per key tile of warpgroup g
-    uint64_t *o_done = pd_full + 2;
-    uint64_t *drain = o_done + 2;
+    // ks_done[s]: the S MMAs of the key tile in K slot s are done, so the slot
+    // may be refilled (and, by columns, the softmax may read S).  vo_done[s]:
+    // the PV MMAs of the key tile in V slot s are done, so the slot may be
+    // refilled (and, by columns, O may be rescaled or read).  By columns one
+    // commit per MMA group thus signals both consumers; neither can fall two
+    // phases behind on a slot, because the next phase needs the slot's next
+    // load, issued by the TMA warp only after its wait, and the MMAs of a key
+    // tile that this softmax warp has not yet written P for.  By tiles the
+    // softmax keeps barriers of its own (s_full[g], o_done[g] for warpgroup
+    // g), which measured faster there.
+    uint64_t *ks_done = k_full + C::NK;
+    uint64_t *v_full = ks_done + C::NK;
+    uint64_t *vo_done = v_full + C::NV;
+    uint64_t *p_full = vo_done + C::NV;  // [2] bf16 P written
+    uint64_t *pd_full = p_full + 2;      // [2] bf16 P (sS' - c) written
+    uint64_t *drain = pd_full + 2;
+    uint64_t *s_full = drain + 1;        // by tiles: [2] S of warpgroup g's key tile written
+    uint64_t *o_done = s_full + 2;       // by tiles: [2] PV of warpgroup g's key tile done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -313,19 +321,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         mbar_init(q_empty, 1);
         for (int s = 0; s < C::NK; ++s) {
             mbar_init(&k_full[s], 1);
-            mbar_init(&k_empty[s], 1);
+            mbar_init(&ks_done[s], 1);
         }
         for (int s = 0; s < C::NV; ++s) {
             mbar_init(&v_full[s], 1);
-            mbar_init(&v_empty[s], 1);
+            mbar_init(&vo_done[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], C::P_ARRIVALS);
             mbar_init(&pd_full[s], C::P_ARRIVALS);
+            if (C::ALT) {
+                mbar_init(&s_full[s], 1);
+                mbar_init(&o_done[s], 1);
+            }
         }
-        mbar_init(&o_done[0], 1);
-        mbar_init(&o_done[1], 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -385,7 +394,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 for (int j = 0; j <= t.nT; ++j) {
                     if (j < t.nT) {
                         const int s = kc % C::NK;
-                        if (kc >= C::NK) ok = wait_bar(&k_empty[s], ((kc / C::NK) - 1) & 1, wc, SITE_K_EMPTY);
+                        if (kc >= C::NK) ok = wait_bar(&ks_done[s], ((kc / C::NK) - 1) & 1, wc, SITE_K_EMPTY);
                         if (!ok) break;
                         uint8_t *dst = smem + C::OFF_K + s * C::KST_BYTES;
                         mbar_arrive_expect_tx(&k_full[s], ZKV ? C::KST_BYTES / 2 : C::KST_BYTES);
@@ -402,7 +411,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                     if (j >= 1) {
                         const int s = vc % C::NV;
-                        if (vc >= C::NV) ok = wait_bar(&v_empty[s], ((vc / C::NV) - 1) & 1, wc, SITE_V_EMPTY);
+                        if (vc >= C::NV) ok = wait_bar(&vo_done[s], ((vc / C::NV) - 1) & 1, wc, SITE_V_EMPTY);
                         if (!ok) break;
                         uint8_t *dst = smem + C::OFF_V + s * C::VST_BYTES;
                         mbar_arrive_expect_tx(&v_full[s], ZKV ? C::VHALF_BYTES : C::VST_BYTES);
@@ -471,8 +480,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 const uint32_t ob = (kk >> 2) * (2 * BN * 128) + (kk & 3) * 32;
                 mma_ss(tS + BN, desc_add(dqd, oa), desc_add(dk, ob), C::IDESC_SD, (!ZKV || kk > 0) ? 1u : 0u);
             }
-            mma_commit(&k_empty[s]);
-            mma_commit(&s_full[gk & 1]);
+            mma_commit(&ks_done[s]);
+            if (C::ALT) mma_commit(&s_full[gk & 1]);
             issued = true;
         };
         // LBO: distance between 64-column blocks of V
@@ -505,8 +514,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             for (int kk = 0; kk < BN / 16; ++kk)  // O'_acc += P(sS' - c) V (with V' = 0 it starts O'_acc)
                 mma_ts(tbase + C::T_OD(ow), tP + C::t_pk(kk, true), desc_add(dv, kk * 2048), C::IDESC_PV,
                        (!ZKV || !first || kk > 0) ? 1u : 0u);
-            mma_commit(&v_empty[s]);
-            mma_commit(&o_done[ow]);
+            mma_commit(&vo_done[s]);
+            if (C::ALT) mma_commit(&o_done[ow]);
         };
         // Fixed order per query tile: S_0, S_1, PV_0, S_2, PV_1, ...: S_{j+1}
         // runs on the tensor core while the softmax works on key tile j, and
@@ -895,7 +904,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 const int gk = gg + j;
                 const int bsel = gk & 1;
                 const uint32_t tS = tbase + lane_off + C::T_S + bsel * (2 * BN);
-                if (!__all_sync(0xffffffffu, wait_bar_fast(&s_full[bsel], (gk >> 1) & 1, wc, SITE_S_FULL))) {
+                if (!__all_sync(0xffffffffu, wait_bar_fast(&ks_done[gk % C::NK], (gk / C::NK) & 1, wc, SITE_S_FULL))) {
                     err = true;
                     if (j == 0) bar_and(BAR_SOFT, NSOFT, false);  // the others wait there at key tile 0
                     break;
@@ -960,9 +969,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
                 if (j >= 1) {
                     // PV of the previous key tile must be done before O may be
-                    // rescaled; every warp observes every phase of o_done in
-                    // order (phase gk needs this warp's P of key tile gk).
-                    if (!__all_sync(0xffffffffu, wait_bar_fast(&o_done[0], (gk - 1) & 1, wc, SITE_O_DONE))) {
+                    // rescaled; a warp cannot fall two phases behind on that V
+                    // slot (the next one needs this warp's P of key tile gk + 1).
+                    if (!__all_sync(0xffffffffu, wait_bar_fast(&vo_done[(gk - 1) % C::NV], ((gk - 1) / C::NV) & 1,
+                                                               wc, SITE_O_DONE))) {
                         err = true;
                         break;
                     }
@@ -1084,7 +1094,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             bool ok;
             {
                 bool done = false;
-                if (!err) done = wait_bar(&o_done[0], (gg + nT - 1) & 1, wc, SITE_O_DONE, true);
+                if (!err) {
+                    const int last = gg + nT - 1;
+                    done = wait_bar(&vo_done[last % C::NV], (last / C::NV) & 1, wc, SITE_O_DONE, true);
+                }
                 ok = bar_and(BAR_SOFT, NSOFT, done);  // reached by all 256 threads
             }
             gg += nT;
