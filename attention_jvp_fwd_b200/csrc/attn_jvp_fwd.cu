@@ -145,6 +145,7 @@ struct Params {
     CUtensorMap tm_q, tm_qd, tm_k, tm_kd, tm_v, tm_vd;
     void *o;
     void *od;
+    int out_v8;  // o and od are 32-byte aligned: the epilogue stores 32 bytes at a time
     float *lse;
     float *lse_dot;  // NULL: not computed
     const int32_t *kv_len;
@@ -171,6 +172,47 @@ enum : int {
     EV_SM_PD = 7,    // softmax: bf16 P (sS' - c) stored and signalled (+ 3g)
     TRACE_EVENTS = 11,
 };
+
+__device__ __forceinline__ void st_global_v8(void *dst, const uint32_t (&v)[8])
+{
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
+// Columns [c, c + 32) of the output rows of a warp, 32 bf16 (64 bytes) per
+// lane in pv; `row` is the lane's own row (row index parity = lane parity),
+// `ok_even` / `ok_odd` whether the even / odd row of its lane pair exists.
+// Each thread owns a row, so a plain store of the warp touches 32 rows.  When
+// the output is 32-byte aligned (v8), lanes 2i and 2i + 1 swap halves: then
+// each 32-byte store lands next to its partner's, and one store of the warp
+// covers 16 rows x 64 contiguous bytes in whole L2 sectors.  Called by all 32
+// lanes (the shuffle); the stores themselves are predicated.
+template <int D>
+__device__ __forceinline__ void store_cols32(__nv_bfloat16 *row, int c, const uint32_t (&pv)[16], bool v8,
+                                             bool odd, bool ok_even, bool ok_odd)
+{
+    if (v8) {
+        uint32_t x[8], a[8], b[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = __shfl_xor_sync(0xffffffffu, odd ? pv[i] : pv[8 + i], 1);
+        // even lane: its first half to its row, the partner's first half to the odd row;
+        // odd lane: the partner's second half to the even row, its second half to its row
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            a[i] = odd ? x[i] : pv[i];
+            b[i] = odd ? pv[8 + i] : x[i];
+        }
+        __nv_bfloat16 *even_row = odd ? row - D : row;
+        const int off = c + (odd ? 16 : 0);
+        if (ok_even) st_global_v8(even_row + off, a);
+        if (ok_odd) st_global_v8(even_row + D + off, b);
+    } else if (odd ? ok_odd : ok_even) {
+        uint4 *d4 = reinterpret_cast<uint4 *>(row + c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pv[4 * i], pv[4 * i + 1], pv[4 * i + 2], pv[4 * i + 3]);
+    }
+}
 
 // One query tile: rows q0 .. q0 + 127 of head bh, against the nb valid keys
 // of its batch (nT key tiles).
@@ -845,15 +887,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                             for (int i = 0; i < 32; ++i) acc[i] = fmaf(wh, u2f(odv[i]), fmaf(kh, u2f(ov[i]), acc[i]));
                         }
                     }
-                    if (grow < p.Lq) {
-                        uint32_t pv[16];
+                    uint32_t pv[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
-                        uint4 *dst = reinterpret_cast<uint4 *>(out_ptr + c);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(pv[4 * i], pv[4 * i + 1], pv[4 * i + 2], pv[4 * i + 3]);
-                    }
+                    for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+                    store_cols32<D>(out_ptr, c, pv, p.out_v8, lane & 1, (grow & ~1) < p.Lq, (grow | 1) < p.Lq);
                 }
                 if (g == 0 && grow < p.Lq) p.lse[lrow] = (M + log2f(lt)) * 0.69314718055994531f;
                 if (g == 1 && p.lse_dot && grow < p.Lq) p.lse_dot[lrow] = mu;
@@ -1132,12 +1169,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         pv[i] = pack_bf16x2(fmaf(-coef, u2f(ov[2 * i]), u2f(odv[2 * i])) * inv_l,
                                             fmaf(-coef, u2f(ov[2 * i + 1]), u2f(odv[2 * i + 1])) * inv_l);
                 }
-                if (grow < p.Lq) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(out_ptr + c);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(pv[4 * i], pv[4 * i + 1], pv[4 * i + 2], pv[4 * i + 3]);
-                }
+                store_cols32<D>(out_ptr, c, pv, p.out_v8, lane & 1, (grow & ~1) < p.Lq, (grow | 1) < p.Lq);
             }
             if (g == 0 && grow < p.Lq) p.lse[lrow] = (m_used + log2f(lt)) * 0.69314718055994531f;
             // lse' = sum_j P_j s S'_j = c + a / l
@@ -1286,6 +1318,7 @@ static int launch(const void *q, const void *k, const void *v, const void *qd, c
         return ATTN_JVP_ERR_LAUNCH;
     prm.o = o;
     prm.od = od;
+    prm.out_v8 = ((reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(od)) & 31u) == 0;
     prm.lse = lse;
     prm.lse_dot = lse_dot;
     prm.kv_len = kv_len;

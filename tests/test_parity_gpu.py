@@ -135,3 +135,25 @@ def test_many_one_row_query_tiles(d):
     CTA walks two or three nearly empty query tiles."""
     w = W.make_custom(2, 150, 3, 700, d, seed=15)
     compare(gpu_rows(*run_gpu(w)), oracle_ref(w), f"one-row tiles d{d}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_outputs_16_byte_aligned(d):
+    """Output buffers that are 16-byte but not 32-byte aligned take the
+    16-byte store path of the epilogue; the results must not change."""
+    w = W.make_custom(2, 2, 200, 300, d, seed=31)
+    ins = [to_dev(x) for x in w.inputs()]
+    n = 2 * 2 * 200 * d
+    base_o = torch.empty(n + 16, dtype=torch.bfloat16, device="cuda")
+    base_od = torch.empty(n + 16, dtype=torch.bfloat16, device="cuda")
+    o = base_o[8:8 + n].view(2, 2, 200, d)     # 8 bf16 = 16 bytes past a 256-byte boundary
+    od = base_od[8:8 + n].view(2, 2, 200, d)
+    assert o.data_ptr() % 32 == 16 and od.data_ptr() % 32 == 16
+    lse = torch.empty((2, 2, 200), dtype=torch.float32, device="cuda")
+    from attention_jvp_fwd_b200 import attn_jvp_fwd
+    attn_jvp_fwd(*ins, scale=w.scale, out=(o, od, lse))
+    torch.cuda.synchronize()
+    compare(gpu_rows(o, od, lse), oracle_ref(w), f"16-byte aligned outputs d{d}")
+    ref = [t.clone() for t in attn_jvp_fwd(*ins, scale=w.scale)]
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref[0]) and torch.equal(od, ref[1]) and torch.equal(lse, ref[2])
