@@ -14,9 +14,11 @@ these pipeline events; a stamp that was not taken stays 0:
 
 Stamps compare only within a CTA (each SM has its own clock).  The summary
 takes medians over key tiles, so the rare epilogue gap between query tiles
-does not dominate.
+does not dominate; ``summarize_boundaries`` measures that gap on its own.
 """
 import numpy as np
+
+BM, BN = 128, 64  # query rows and keys per tile
 
 K_LOAD, V_LOAD, S_ISSUE, PA_ISSUE, PB_ISSUE = 0, 1, 2, 3, 4
 SM_S, SM_P, SM_PD = 5, 6, 7
@@ -76,6 +78,46 @@ def summarize(trace, skip: int = 2) -> dict:
     return {k: float(np.median(v)) if v else float("nan") for k, v in out.items()}
 
 
+def query_tile_starts(B: int, H: int, Lq: int, Lk: int, kv_len, grid: int, cta: int) -> list:
+    """(first key tile, key tiles) of each query tile that CTA ``cta`` walks,
+    in its own key-tile count, the way the kernel walks them: query tiles
+    w = cta, cta + grid, ... of the ceil(Lq / 128) * B * H tiles, the query
+    tile varying fastest, tiles without keys skipped.  ``kv_len`` is None or a
+    sequence of B key lengths (clamped to [0, Lk])."""
+    nqt = (Lq + BM - 1) // BM
+    starts, gk = [], 0
+    for w in range(cta, nqt * B * H, grid):
+        b = (w // nqt) // H
+        nb = Lk if kv_len is None else min(max(int(kv_len[b]), 0), Lk)
+        nt = (nb + BN - 1) // BN
+        if nt == 0:
+            continue
+        starts.append((gk, nt))
+        gk += nt
+    return starts
+
+
+def summarize_boundaries(trace, starts_per_cta) -> dict:
+    """Median clocks from the last P (sS' - c) signal of a query tile to the
+    first S seen of the CTA's next query tile (the epilogue and the refill
+    between them), over the boundaries whose stamps are in the trace.
+    ``starts_per_cta[c]`` is ``query_tile_starts`` for CTA c."""
+    t = np.asarray(trace, dtype=np.int64)
+    gaps = []
+    for c, starts in enumerate(starts_per_cta[: t.shape[0]]):
+        tc = t[c]
+        for (g0, n0), (g1, _) in zip(starts, starts[1:]):
+            last = g0 + n0 - 1
+            if g1 >= tc.shape[0]:
+                break
+            pd = [tc[last, _sm(g, SM_PD)] for g in (0, 1) if tc[last, _sm(g, SM_PD)]]
+            seen = [tc[g1, _sm(g, SM_S)] for g in (0, 1) if tc[g1, _sm(g, SM_S)]]
+            if pd and seen:
+                gaps.append(min(seen) - max(pd))
+    return {"boundaries": len(gaps),
+            "epilogue_gap": float(np.median(gaps)) if gaps else float("nan")}
+
+
 def format_summary(s: dict) -> str:
     return "\n".join(f"{k:14s} {v:10.0f} cycles" for k, v in s.items())
 
@@ -114,7 +156,15 @@ def main(argv=None):
         raise SystemExit(f"device status {st} at site {site}")
     print(f"{w.name}: B={w.B} H={w.H} Lq={w.Lq} Lk={w.Lk} d={w.d}; {tr.shape[0]} CTAs x "
           f"{tr.shape[1]} key tiles stamped")
-    print(format_summary(summarize(tr.cpu().numpy())))
+    t = tr.cpu().numpy()
+    print(format_summary(summarize(t)))
+    n_tiles = ((w.Lq + BM - 1) // BM) * w.B * w.H
+    grid = min(n_tiles, torch.cuda.get_device_properties(dev).multi_processor_count)
+    starts = [query_tile_starts(w.B, w.H, w.Lq, w.Lk, w.kv_len, grid, c) for c in range(t.shape[0])]
+    bs = summarize_boundaries(t, starts)
+    if bs["boundaries"]:
+        print(f"{'epilogue_gap':14s} {bs['epilogue_gap']:10.0f} cycles  (last P(sS'-c) of a query "
+              f"tile -> first S seen of the next; {bs['boundaries']} boundaries)")
     return 0
 
 

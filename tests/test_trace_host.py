@@ -51,3 +51,54 @@ def test_missing_stamps_and_shape_check():
     assert all(math.isnan(v) for v in s.values())
     with pytest.raises(ValueError):
         T.summarize(np.zeros((1, 4, 5), np.int64))
+
+
+@pytest.mark.parametrize("B,H,Lq,Lk,kv,grid", [
+    (2, 1, 256, 100, [0, 100], 3),
+    (4, 3, 1000, 512, [421, 81, 0, 600], 7),
+    (1, 24, 4099, 4099, None, 148),
+])
+def test_query_tile_starts_follow_the_kernel_walk(B, H, Lq, Lk, kv, grid):
+    """Every query tile in launch order goes to CTA w % grid; a CTA's key tiles
+    are counted over its own query tiles, skipping those without keys."""
+    nqt = -(-Lq // 128)
+    expect = {c: [] for c in range(grid)}
+    count = {c: 0 for c in range(grid)}
+    for w in range(nqt * B * H):
+        b = w // (nqt * H)
+        nb = Lk if kv is None else min(max(kv[b], 0), Lk)
+        nt = -(-nb // 64)
+        if nt:
+            expect[w % grid].append((count[w % grid], nt))
+            count[w % grid] += nt
+    for c in range(grid):
+        assert T.query_tile_starts(B, H, Lq, Lk, kv, grid, c) == expect[c]
+
+
+@pytest.mark.parametrize("alt", [False, True])
+def test_boundary_gap(alt):
+    """Query tiles of 3, 2 and 4 key tiles on one CTA; the gaps from the last
+    P (sS' - c) of one query tile to the first S seen of the next are 900 and
+    1500, so the median of the two is 1200."""
+    starts = [[(0, 3), (3, 2), (5, 4)]]
+    t = np.zeros((1, 9, T.EVENTS), np.int64)
+    clock = 1000
+    for i in range(9):
+        if i == 3:
+            clock += 900
+        if i == 5:
+            clock += 1500
+        gs = [i % 2] if alt else [0, 1]
+        for g in gs:
+            t[0, i, T.SM_S + 3 * g] = clock
+            t[0, i, T.SM_PD + 3 * g] = clock + 2000 - 5 * g
+        clock += 2000
+    r = T.summarize_boundaries(t, starts)
+    assert r["boundaries"] == 2 and r["epilogue_gap"] == 1200
+
+
+def test_boundary_gap_outside_the_stamped_range():
+    starts = [[(0, 3), (3, 2)]]
+    t = np.zeros((1, 3, T.EVENTS), np.int64)  # only the first query tile is stamped
+    r = T.summarize_boundaries(t, starts)
+    assert r["boundaries"] == 0 and math.isnan(r["epilogue_gap"])
