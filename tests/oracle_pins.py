@@ -295,6 +295,9 @@ def pin_hand_examples(lib):
         assert np.array_equal(np.isneginf(lse), np.isneginf(el)), c["name"]
         fin = np.isfinite(el)
         assert np.allclose(lse[fin], el[fin], rtol=1e-14, atol=1e-14), c["name"]
+        if "lse_dot" in c:  # lse' = sum_j P_j S'_j, worked out by hand as well
+            mu = run_mu(lib, *ins, c["scale"], kv_len=kv)[3]
+            assert np.allclose(mu, _golden_array(c["lse_dot"]), rtol=1e-14, atol=1e-14), c["name"]
 
 
 def run_mu(lib, q, k, v, qd, kd, vd, scale, kv_len=None, rows=None):
