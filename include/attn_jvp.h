@@ -66,7 +66,10 @@ typedef enum {
  *
  *   q, k, v              bf16 device pointers (layout above)
  *   q_dot, k_dot, v_dot  bf16 device pointers, the tangents Q', K', V'
- *   o, o_dot             bf16 device pointers, written
+ *   o, o_dot             bf16 device pointers, written.  When both are 32-byte
+ *                        aligned (as cudaMalloc and PyTorch allocations are), the
+ *                        epilogue stores 32 bytes at a time; 16-byte aligned
+ *                        outputs take a slower store path with the same results
  *   lse                  fp32 device pointer, written (natural log)
  *   B, H, Lq, Lk         >= 1; B*H*Lq and B*H*Lk below 2^31; Lq, Lk below 2^31
  *   d                    64 or 128
