@@ -25,8 +25,8 @@ ATTN_JVP_ERR_TIMEOUT = -6
 ATTN_JVP_ERR_VALUE = -7
 ATTN_JVP_DEBUG_STARVE_Q = 1
 
-EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_ex", "attn_jvp_fwd_debug", "attn_jvp_fwd_trace",
-            "attn_jvp_check", "attn_jvp_status_string", "attn_jvp_version", "scm_tangent_loss",
+EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_ex", "attn_jvp_fwd_ws", "attn_jvp_workspace_bytes",
+            "attn_jvp_fwd_debug", "attn_jvp_fwd_trace", "attn_jvp_check", "attn_jvp_status_string", "attn_jvp_version", "scm_tangent_loss",
             "qkv_rmsnorm_jvp", "qkv_prologue_check")
 TRACE_EVENTS = 11  # stamps per key tile of attn_jvp_fwd_trace
 
@@ -66,6 +66,10 @@ def load_library():
             lib.scm_tangent_loss.argtypes = [vp] * 5 + [i32, ctypes.c_longlong, f32, vp]
             lib.attn_jvp_fwd_ex.restype = i32
             lib.attn_jvp_fwd_ex.argtypes = [vp] * 10 + [i32] * 5 + [f32, vp, vp]
+            lib.attn_jvp_fwd_ws.restype = i32
+            lib.attn_jvp_fwd_ws.argtypes = [vp] * 10 + [i32] * 5 + [f32, vp, vp, ctypes.c_size_t, vp]
+            lib.attn_jvp_workspace_bytes.restype = ctypes.c_size_t
+            lib.attn_jvp_workspace_bytes.argtypes = [i32] * 5
             lib.attn_jvp_fwd_debug.restype = i32
             lib.attn_jvp_fwd_debug.argtypes = [vp] * 9 + [i32] * 5 + [f32, vp, vp,
                                                                      ctypes.c_uint64, i32]
@@ -119,8 +123,17 @@ def _stream_handle(device, stream):
     return ctypes.c_void_p(int(stream.cuda_stream))
 
 
+def attn_jvp_workspace_bytes(B: int, H: int, Lq: int, Lk: int, d: int, device=None) -> int:
+    """Workspace bytes the split call needs for this shape on `device` (0: no
+    split for this shape)."""
+    device = device if device is not None else torch.cuda.current_device()
+    with torch.cuda.device(device):
+        return int(load_library().attn_jvp_workspace_bytes(int(B), int(H), int(Lq), int(Lk), int(d)))
+
+
 def attn_jvp_fwd(q, k, v, q_dot, k_dot, v_dot, scale: float | None = None, kv_len=None,
-                 out=None, stream=None, *, lse_dot: bool = False,
+                 out=None, stream=None, *, lse_dot: bool = False, split: bool = True,
+                 workspace: torch.Tensor | None = None,
                  _debug_timeout_ns: int | None = None, _debug_flags: int = 0):
     """O = softmax(scale Q K^T) V, its tangent O' along (Q', K', V'), and lse.
 
@@ -132,6 +145,11 @@ def attn_jvp_fwd(q, k, v, q_dot, k_dot, v_dot, scale: float | None = None, kv_le
     ``out`` may supply (o, o_dot, lse[, lse_dot]) buffers.  Queued on
     ``stream`` (default: the current stream).  Returns (o, o_dot, lse) or
     (o, o_dot, lse, lse_dot), lse and lse_dot fp32 [B, H, Lq].
+
+    ``split`` (default) cuts the last wave of query tiles into key ranges
+    (attn_jvp_fwd_ws); its workspace is ``workspace`` (a uint8 CUDA tensor of
+    at least attn_jvp_workspace_bytes bytes) or, if None, allocated here.
+    ``split=False`` walks every query tile whole and needs no workspace.
     """
     B, H, Lq, Lk, d = _check_inputs(q, k, v, q_dot, k_dot, v_dot)
     if scale is None:
@@ -174,6 +192,18 @@ def attn_jvp_fwd(q, k, v, q_dot, k_dot, v_dot, scale: float | None = None, kv_le
                 raise ValueError("the debug entry point takes all six inputs and no lse_dot")
             rc = lib.attn_jvp_fwd_debug(*ptrs, B, H, Lq, Lk, d, float(scale), kv_ptr, sh,
                                         int(_debug_timeout_ns or 0), int(_debug_flags))
+        elif split:
+            need = int(lib.attn_jvp_workspace_bytes(B, H, Lq, Lk, d))
+            ws = workspace
+            if need and ws is None:
+                ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+                if stream is not None:
+                    ws.record_stream(stream)  # alive until the kernel on `stream` is done
+            if ws is not None and (ws.dtype != torch.uint8 or ws.device != q.device
+                                   or not ws.is_contiguous()):
+                raise ValueError("workspace must be a contiguous uint8 tensor on q's device")
+            rc = lib.attn_jvp_fwd_ws(*ptrs, ptr(ld), B, H, Lq, Lk, d, float(scale), kv_ptr,
+                                     ptr(ws), 0 if ws is None else ws.numel(), sh)
         elif k_dot is None or lse_dot:
             rc = lib.attn_jvp_fwd_ex(*ptrs, ptr(ld), B, H, Lq, Lk, d, float(scale), kv_ptr, sh)
         else:

@@ -28,8 +28,9 @@
 // events into a caller buffer; it computes the same results.
 //
 // c is a per-row constant (the p-weighted mean of s S'_raw over the first 32
-// keys).  In exact arithmetic O' does not depend on it; it keeps the bf16
-// products P (sS' - c) small when S' has a large row mean.
+// keys, or 0 when all their p underflow).  In exact arithmetic O' does not
+// depend on it; it keeps the bf16 products P (sS' - c) small when S' has a
+// large row mean.
 //
 // Every wait on an mbarrier is bounded (default 2 s, wall clock); a wait that
 // runs out records a site code in a device status word, tells the other
@@ -157,7 +158,24 @@ struct Params {
     // trace build only: clock64 stamps [trace_ctas][trace_tiles][TRACE_EVENTS]
     unsigned long long *trace;
     int trace_tiles, trace_ctas;
+    // Last-wave key split.  The first n_full query tiles are walked whole,
+    // round robin over the CTAs (n_full is a multiple of the grid when
+    // there is a split).  The remaining tiles are each cut into split_S key
+    // ranges, and CTA u < n_units takes unit u after its whole tiles: tile
+    // n_full + u / split_S, range u % split_S.  A range writes its partial
+    // softmax state to part[u]; the last range of a tile to finish (counted
+    // in cnt[u / split_S], zeroed before the launch) merges them.
+    int n_full, split_S, n_units;
+    float *part;
+    int *cnt;
 };
+
+// Floats of one partial record per query row: m (log2 units), l, a, c, then
+// the unnormalised O_acc and O'_acc rows.  A record holds 128 rows with the
+// row index fastest, so a warp's loads and stores of one field coalesce.
+template <int D>
+__host__ __device__ constexpr int part_fields() { return 4 + 2 * D; }
+constexpr int SPLIT_MAX = 8;  // ranges per split tile at most
 
 // Events a trace build stamps for each of a CTA's key tiles (gg counts the
 // key tiles of all the CTA's query tiles), in SM clock cycles.
@@ -214,26 +232,71 @@ __device__ __forceinline__ void store_cols32(__nv_bfloat16 *row, int c, const ui
     }
 }
 
-// One query tile: rows q0 .. q0 + 127 of head bh, against the nb valid keys
-// of its batch (nT key tiles).
+// One work item: rows q0 .. q0 + 127 of head bh, against key tiles
+// [jb, jb + nT) of the nb valid keys of its batch (the whole tile has
+// ceil(nb / BN) key tiles; a split tile's range has fewer).  part < 0: the
+// outputs are written directly; part >= 0: the partial state goes to record
+// `part`, and the range is one of nseg of split tile `tsplit`.
 struct Tile {
-    int q0, bh, nb, nT;
+    int q0, bh, nb, jb, nT;
+    int part, tsplit, nseg;
 };
 
-__device__ __forceinline__ Tile tile_of(const Params &p, int w)
+enum : int { ITEM_END = 0, ITEM_WORK = 1, ITEM_SKIP = 2 };
+
+// The k-th work item of this CTA.  Every role walks the same sequence.
+__device__ __forceinline__ int item_of(const Params &p, int k, Tile &t)
 {
-    Tile t;
+    const int b = blockIdx.x, G = gridDim.x;
+    const int nk_full = b < p.n_full ? (p.n_full - 1 - b) / G + 1 : 0;
+    int w, seg = 0, S = 1;
+    if (k < nk_full) {
+        w = b + k * G;
+    } else if (k == nk_full && b < p.n_units) {
+        w = p.n_full + b / p.split_S;
+        seg = b % p.split_S;
+        S = p.split_S;
+    } else {
+        return ITEM_END;
+    }
     const int qt = w % p.nqt;  // query tile fastest: CTAs running together share K/V in L2
     t.bh = w / p.nqt;
     t.q0 = qt * BM;
     int nb = p.Lk;
     if (p.kv_len) nb = min(max(p.kv_len[t.bh / p.H], 0), p.Lk);
     t.nb = nb;
-    t.nT = (nb + BN - 1) / BN;
-    return t;
+    const int nT = (nb + BN - 1) / BN;
+    t.jb = 0;
+    t.nT = nT;
+    t.part = -1;
+    t.tsplit = 0;
+    t.nseg = 1;
+    if (S > 1) {
+        // a tile with fewer key tiles than ranges uses fewer ranges; one
+        // without keys is written (as zeros) by its range 0 alone
+        const int se = min(S, nT);
+        if (seg >= max(se, 1)) return ITEM_SKIP;
+        if (se > 1) {
+            t.jb = seg * nT / se;
+            t.nT = (seg + 1) * nT / se - t.jb;
+            t.part = b;
+            t.tsplit = b / S;
+            t.nseg = se;
+        }
+    }
+    return ITEM_WORK;
 }
 
 __device__ int g_status;  // first wait site that gave up since the last check
+__device__ int g_status_taken;  // the word as the last check took it
+
+// Read and clear the status word in one atomic step, ordered on the checking
+// stream, so a site recorded by a kernel on another stream between a read
+// and a clear cannot be lost.
+__global__ void take_status_kernel() { g_status_taken = atomicExch(&g_status, 0); }
+
+// Host threads that check at the same time take turns on g_status_taken.
+static std::mutex g_check_mu;
 
 struct WaitCtx {
     volatile int *abort;
@@ -298,6 +361,91 @@ __device__ __forceinline__ float row_max64(const uint32_t (&a)[32], const uint32
 __device__ __forceinline__ float row_min64(const uint32_t (&a)[32], const uint32_t (&b)[32])
 {
     return row_ext64<true>(a, b);
+}
+
+// ---- last-wave key split: partial records and their merge
+
+template <int D>
+__device__ __forceinline__ float *part_field(const Params &p, int u, int f)
+{
+    return p.part + (static_cast<size_t>(u) * part_fields<D>() + f) * BM;
+}
+
+template <int D>
+__device__ __forceinline__ void part_put_scalars(const Params &p, int u, int r, float m, float l, float a, float c)
+{
+    part_field<D>(p, u, 0)[r] = m;
+    part_field<D>(p, u, 1)[r] = l;
+    part_field<D>(p, u, 2)[r] = a;
+    part_field<D>(p, u, 3)[r] = c;
+}
+
+// Columns [c, c + 32) of O_acc (which = 0) or O'_acc (which = 1).
+template <int D>
+__device__ __forceinline__ void part_put_cols(const Params &p, int u, int r, int which, int c, const float (&v)[32])
+{
+#pragma unroll
+    for (int i = 0; i < 32; ++i) part_field<D>(p, u, 4 + which * D + c + i)[r] = v[i];
+}
+
+// Called by all 256 softmax threads after they wrote this range's partial
+// record.  The range that finishes last (a counter per split tile, zeroed
+// before the launch) merges the records of all ranges of the tile, with
+// M = max m_s, b_s = 2^(m_s - M), L = sum b_s l_s:
+//   mu = sum b_s (a_s + c_s l_s) / L,  O = sum b_s O_s / L,
+//   O' = sum b_s (O'_s + (c_s - mu) O_s) / L,  lse = (M + log2 L) ln 2,
+// and writes the outputs (warpgroup 0: O and lse, warpgroup 1: O' and lse').
+// No CTA waits for another: the ranges that finish earlier just leave.
+template <int D>
+__device__ __noinline__ void split_finish(const Params &p, const Tile &t, int g, int r, int lane, __nv_bfloat16 *out_ptr,
+                             int grow, size_t lrow, uint8_t *flag_smem)
+{
+    volatile int *flag = reinterpret_cast<volatile int *>(flag_smem);
+    __threadfence();  // this thread's record stores, before the count
+    bar_sync(BAR_SOFT, NSOFT);
+    if (threadIdx.x == 64) *flag = atomicAdd(&p.cnt[t.tsplit], 1) == t.nseg - 1;
+    bar_sync(BAR_SOFT, NSOFT);
+    const bool last = *flag != 0;
+    bar_sync(BAR_SOFT, NSOFT);  // everyone has read the flag before it can be reused
+    if (!last) return;
+    __threadfence();
+    const int u0 = t.tsplit * p.split_S;
+    float M = -INFINITY;
+    for (int s = 0; s < t.nseg; ++s) M = fmaxf(M, __ldcg(part_field<D>(p, u0 + s, 0) + r));
+    float L = 0.f, num = 0.f;
+    for (int s = 0; s < t.nseg; ++s) {
+        const float b = ex2_approx(__ldcg(part_field<D>(p, u0 + s, 0) + r) - M);
+        const float ls = __ldcg(part_field<D>(p, u0 + s, 1) + r);
+        L = fmaf(b, ls, L);
+        num = fmaf(b, fmaf(__ldcg(part_field<D>(p, u0 + s, 3) + r), ls, __ldcg(part_field<D>(p, u0 + s, 2) + r)), num);
+    }
+    const float inv_l = 1.f / L;
+    const float mu = num * inv_l;
+#pragma unroll 1
+    for (int c = 0; c < D; c += 32) {
+        float acc[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+        for (int s = 0; s < t.nseg; ++s) {
+            const float w = ex2_approx(__ldcg(part_field<D>(p, u0 + s, 0) + r) - M) * inv_l;
+            const float *o = part_field<D>(p, u0 + s, 4 + c) + r;
+            if (g == 0) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, __ldcg(o + i * BM), acc[i]);
+            } else {
+                const float kk = w * (__ldcg(part_field<D>(p, u0 + s, 3) + r) - mu);
+                const float *od = part_field<D>(p, u0 + s, 4 + D + c) + r;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, __ldcg(od + i * BM), fmaf(kk, __ldcg(o + i * BM), acc[i]));
+            }
+        }
+        uint32_t pv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+        store_cols32<D>(out_ptr, c, pv, p.out_v8, lane & 1, (grow & ~1) < p.Lq, (grow | 1) < p.Lq);
+    }
+    if (g == 0 && grow < p.Lq) p.lse[lrow] = (M + log2f(L)) * 0.69314718055994531f;
+    if (g == 1 && p.lse_dot && grow < p.Lq) p.lse_dot[lrow] = mu;
 }
 
 // ZKV: K' = V' = 0 (frozen keys and values, e.g. text tokens).  Then S'_raw
@@ -415,9 +563,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             int nq = 0;           // Q loads issued
             int kc = 0, vc = 0;   // K and V loads issued
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < p.n_tiles; w += gridDim.x) {
-                const Tile t = tile_of(p, w);
-                if (t.nT == 0) continue;
+            Tile t;
+            for (int k = 0; ok; ++k) {
+                const int it = item_of(p, k, t);
+                if (it == ITEM_END) break;
+                if (it == ITEM_SKIP || t.nT == 0) continue;
                 if (lc >= 1 && !wait_bar(q_empty, (lc - 1) & 1, wc, SITE_Q_EMPTY)) {
                     ok = false;
                     break;
@@ -442,11 +592,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         mbar_arrive_expect_tx(&k_full[s], ZKV ? C::KST_BYTES / 2 : C::KST_BYTES);
 #pragma unroll
                         for (int c = 0; c < C::NKB; ++c) {
-                            tma_load_3d(dst + c * (2 * BN * 128), &p.tm_k, &k_full[s], c * 64, j * BN, t.bh,
-                                        pol_kv);
+                            tma_load_3d(dst + c * (2 * BN * 128), &p.tm_k, &k_full[s], c * 64, (t.jb + j) * BN,
+                                        t.bh, pol_kv);
                             if (!ZKV)
                                 tma_load_3d(dst + c * (2 * BN * 128) + BN * 128, &p.tm_kd, &k_full[s], c * 64,
-                                            j * BN, t.bh, pol_kv);
+                                            (t.jb + j) * BN, t.bh, pol_kv);
                         }
                         stamp(kc, EV_K_LOAD);
                         ++kc;
@@ -459,11 +609,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         mbar_arrive_expect_tx(&v_full[s], ZKV ? C::VHALF_BYTES : C::VST_BYTES);
 #pragma unroll
                         for (int c = 0; c < C::NKB; ++c) {
-                            tma_load_3d(dst + c * (BN * 128), &p.tm_v, &v_full[s], c * 64, (j - 1) * BN, t.bh,
-                                        pol_kv);
+                            tma_load_3d(dst + c * (BN * 128), &p.tm_v, &v_full[s], c * 64, (t.jb + j - 1) * BN,
+                                        t.bh, pol_kv);
                             if (!ZKV)
                                 tma_load_3d(dst + (C::NKB + c) * (BN * 128), &p.tm_vd, &v_full[s], c * 64,
-                                            (j - 1) * BN, t.bh, pol_kv);
+                                            (t.jb + j - 1) * BN, t.bh, pol_kv);
                         }
                         stamp(vc, EV_V_LOAD);
                         ++vc;
@@ -568,9 +718,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         // which the softmax warps write only after their epilogue has read O.
         bool ok = true;
         int lc = 0, gg = 0;
-        for (int w = blockIdx.x; ok && w < p.n_tiles; w += gridDim.x) {
-            const Tile t = tile_of(p, w);
-            if (t.nT == 0) continue;
+        Tile t;
+        for (int k = 0; ok; ++k) {
+            const int it = item_of(p, k, t);
+            if (it == ITEM_END) break;
+            if (it == ITEM_SKIP || t.nT == 0) continue;
             ok = wait_u(q_full, lc & 1, SITE_Q_FULL);
             ++lc;
             if (ok) ok = wait_u(&k_full[gg % C::NK], (gg / C::NK) & 1, SITE_K_FULL);
@@ -625,8 +777,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         if constexpr (C::ALT) {
             int gg = 0;
             const uint32_t tS = tbase + lane_off + C::T_S + g * (2 * BN);  // this warpgroup's S buffer
-            for (int w = blockIdx.x; w < p.n_tiles; w += gridDim.x) {
-                const Tile t = tile_of(p, w);
+            Tile t;
+            for (int k = 0;; ++k) {
+                const int itk = item_of(p, k, t);
+                if (itk == ITEM_END) break;
+                if (itk == ITEM_SKIP) continue;
                 const int grow = t.q0 + r;
                 __nv_bfloat16 *out_ptr =
                     static_cast<__nv_bfloat16 *>(g == 0 ? p.o : p.od) + (static_cast<size_t>(t.bh) * p.Lq + grow) * D;
@@ -655,7 +810,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                     if (tracer) stamp(gk, EV_SM_S + 3 * g);
                     tc_fence_after();
-                    const int vt = nb - j * BN;  // valid keys in the tile
+                    const int vt = nb - (t.jb + j) * BN;  // valid keys in the tile
                     const bool tail = vt < BN;
                     uint32_t ra[32], rb[32];
                     tmem_ld32(tS, ra);       // S, keys 0..31
@@ -775,8 +930,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     tmem_ld_wait(rd);
                     if (nown == 0) {
                         // centring constant c: the p-weighted mean of s S' over
-                        // keys 0..31 of this warpgroup's first key tile (key 0
-                        // is always valid)
+                        // keys 0..31 of this warpgroup's first key tile.  Their
+                        // p can all be 0 (the tile's max among keys 32..63 and
+                        // keys 0..31 more than ~87 logits below it); c cancels
+                        // exactly, so any finite value is right, and 0 is taken.
                         float n0 = 0.f, n1 = 0.f, w0 = 0.f, w1 = 0.f;
 #pragma unroll
                         for (int i = 0; i < 32; i += 2) {
@@ -785,7 +942,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                             w0 += x[i];
                             w1 += x[i + 1];
                         }
-                        cctr = (n0 + n1) / (w0 + w1);
+                        const float wsum = w0 + w1;
+                        cctr = wsum > 0.f ? (n0 + n1) / wsum : 0.f;
                     }
                     uint32_t re[32];
                     tmem_ld32(tS + BN + 32, re);  // S'_raw, keys 32..63
@@ -862,8 +1020,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 const float lt = (has0 ? b0 * l0 : 0.f) + (has1 ? b1 * l1 : 0.f);
                 const float inv_l = 1.f / lt;
                 const float mu = ((has0 ? b0 * fmaf(c0v, l0, a0v) : 0.f) + (has1 ? b1 * fmaf(c1v, l1, a1v) : 0.f)) * inv_l;
-                const float w0 = b0 * inv_l, w1 = b1 * inv_l;
+                // A key range of a split tile keeps its state unnormalised:
+                // m = M, l = L, c = mu, a = 0, O = sum_h b_h O_h and
+                // O' = sum_h b_h (O'_h + (c_h - mu) O_h).
+                const bool part = t.part >= 0;
+                const float wn = part ? 1.f : inv_l;
+                const float w0 = b0 * wn, w1 = b1 * wn;
                 const float k0 = w0 * (c0v - mu), k1 = w1 * (c1v - mu);
+                if (part && g == 0) part_put_scalars<D>(p, t.part, r, M, lt, 0.f, mu);
 #pragma unroll 1
                 for (int c = 0; c < D; c += 32) {
                     float acc[32];
@@ -887,13 +1051,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                             for (int i = 0; i < 32; ++i) acc[i] = fmaf(wh, u2f(odv[i]), fmaf(kh, u2f(ov[i]), acc[i]));
                         }
                     }
+                    if (part) {
+                        part_put_cols<D>(p, t.part, r, g, c, acc);
+                        continue;
+                    }
                     uint32_t pv[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
                     store_cols32<D>(out_ptr, c, pv, p.out_v8, lane & 1, (grow & ~1) < p.Lq, (grow | 1) < p.Lq);
                 }
-                if (g == 0 && grow < p.Lq) p.lse[lrow] = (M + log2f(lt)) * 0.69314718055994531f;
-                if (g == 1 && p.lse_dot && grow < p.Lq) p.lse_dot[lrow] = mu;
+                if (part) {
+                    split_finish<D>(p, t, g, r, lane, out_ptr, grow, lrow, smem + C::OFF_MISC + 8);
+                } else {
+                    if (g == 0 && grow < p.Lq) p.lse[lrow] = (M + log2f(lt)) * 0.69314718055994531f;
+                    if (g == 1 && p.lse_dot && grow < p.Lq) p.lse_dot[lrow] = mu;
+                }
                 // Both warpgroups read O_0 and O_1 above; the next query tile's
                 // first P (after which the MMAs restart an accumulator) comes
                 // from one warpgroup only, so meet here first.  This also
@@ -908,8 +1080,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         // the next query tile while warpgroup 1 still reads the l, a of this one.
         const int c0 = 32 * g;
         int gg = 0;
-        for (int w = blockIdx.x; w < p.n_tiles; w += gridDim.x) {
-            const Tile t = tile_of(p, w);
+        Tile t;
+        for (int k = 0;; ++k) {
+            const int itk = item_of(p, k, t);
+            if (itk == ITEM_END) break;
+            if (itk == ITEM_SKIP) continue;
             const int grow = t.q0 + r;
             const size_t orow = (static_cast<size_t>(t.bh) * p.Lq + grow) * D;
             __nv_bfloat16 *out_ptr = static_cast<__nv_bfloat16 *>(g == 0 ? p.o : p.od) + orow;
@@ -948,7 +1123,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 }
                 if (tracer) stamp(gk, EV_SM_S + 3 * g);
                 tc_fence_after();
-                const int vt = nb - j * BN;  // valid keys in the tile
+                const int vt = nb - (t.jb + j) * BN;  // valid keys in the tile
                 const int valid = vt - c0;   // valid columns of this half
                 const bool tail = vt < BN;
                 float mx;
@@ -1085,7 +1260,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                             w0 += x[i];
                             w1 += x[i + 1];
                         }
-                        cctr = (n0 + n1) / (w0 + w1);
+                        // all p of keys 0..31 can be 0 (the max among keys
+                        // 32..63, keys 0..31 far below it): c cancels exactly,
+                        // so any finite value is right, and 0 is taken
+                        const float wsum = w0 + w1;
+                        cctr = wsum > 0.f ? (n0 + n1) / wsum : 0.f;
                         xch[512 + r] = cctr;
                     }
                     if (!bar_and(BAR_SOFT, NSOFT, true)) {
@@ -1150,6 +1329,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const float coef = (xch[256 + r] + xch[384 + r]) * inv_l;
             const uint32_t to = tbase + lane_off + C::T_O(0);
             const uint32_t tod = tbase + lane_off + C::T_OD(0);
+            if (t.part >= 0) {
+                // a key range of a split tile: its unnormalised state
+                if (g == 0) part_put_scalars<D>(p, t.part, r, m_used, lt, xch[256 + r] + xch[384 + r], cctr);
+#pragma unroll 1
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t v[32];
+                    tmem_ld32((g == 0 ? to : tod) + c, v);
+                    tmem_ld_wait(v);
+                    float acc[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[i] = u2f(v[i]);
+                    part_put_cols<D>(p, t.part, r, g, c, acc);
+                }
+                split_finish<D>(p, t, g, r, lane, out_ptr, grow, lrow, smem + C::OFF_MISC + 8);
+                continue;
+            }
 #pragma unroll 1
             for (int c = 0; c < D; c += 32) {
                 uint32_t ov[32], odv[32];
@@ -1251,13 +1446,63 @@ static int prepare_device(int dev, int *n_sm)
     return ATTN_JVP_OK;
 }
 
+// SM count of the current device (queried once per device).
+static int device_sms(int *n_sm)
+{
+    static std::mutex mu;
+    static int sms[MAX_DEVICES] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return ATTN_JVP_ERR_LAUNCH;
+    std::lock_guard<std::mutex> g(mu);
+    if (sms[dev] == 0 &&
+        (cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms[dev] < 1)) {
+        sms[dev] = 0;
+        return ATTN_JVP_ERR_LAUNCH;
+    }
+    *n_sm = sms[dev];
+    return ATTN_JVP_OK;
+}
+
+// How the last wave of query tiles is cut into key ranges.  With T query
+// tiles on n_sm persistent CTAs, the first floor(T / n_sm) waves are walked
+// whole and the R = T mod n_sm tiles left over are each cut into
+// S = min(n_sm / R, key tiles, SPLIT_MAX) ranges, one per CTA, so the last
+// wave takes about 1/S of a tile's time instead of a whole one.  No split
+// when S < 2 (the last wave is nearly full, or a tile has one key tile).
+struct SplitPlan {
+    int grid = 0, n_full = 0, S = 0, n_units = 0, n_split_tiles = 0;
+    size_t cnt_bytes = 0, bytes = 0;
+};
+
+static SplitPlan split_plan(long long T, int n_sm, int Lk, int d)
+{
+    SplitPlan sp;
+    sp.grid = static_cast<int>(T < n_sm ? T : n_sm);
+    sp.n_full = static_cast<int>(T);
+    const long long nf = T / n_sm * n_sm;
+    const int R = static_cast<int>(T - nf);
+    const int nT = (Lk + BN - 1) / BN;
+    int S = R ? n_sm / R : 0;
+    S = S < nT ? S : nT;
+    S = S < SPLIT_MAX ? S : SPLIT_MAX;
+    if (S >= 2) {
+        sp.grid = n_sm;
+        sp.n_full = static_cast<int>(nf);
+        sp.S = S;
+        sp.n_units = R * S;
+        sp.n_split_tiles = R;
+        sp.cnt_bytes = (static_cast<size_t>(R) * 4 + 255) / 256 * 256;
+        sp.bytes = sp.cnt_bytes + static_cast<size_t>(sp.n_units) * (4 + 2 * d) * BM * 4;
+    }
+    return sp;
+}
+
 template <int D, bool ZKV, bool TRACE = false>
-static int launch_kernel(const Params &prm, cudaStream_t s)
+static int launch_kernel(const Params &prm, int grid, cudaStream_t s)
 {
     int dev = 0, n_sm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     if (int rc = prepare_device<D, ZKV, TRACE>(dev, &n_sm)) return rc;
-    const int grid = prm.n_tiles < n_sm ? prm.n_tiles : n_sm;
     attn_jvp_fwd_kernel<D, ZKV, TRACE><<<grid, NTHREADS, Cfg<D>::SMEM_BYTES, s>>>(prm);
     return ATTN_JVP_OK;
 }
@@ -1270,11 +1515,14 @@ static bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb)
 
 // allow_zero_kv: k_dot and v_dot may both be NULL (K' = V' = 0).
 // trace != NULL: the trace build, stamping [trace_ctas][trace_tiles][TRACE_EVENTS].
+// workspace != NULL: the last-wave key split, with its records and counters
+// in workspace (workspace_bytes at least what split_plan asks for).
 static int launch(const void *q, const void *k, const void *v, const void *qd, const void *kd,
                   const void *vd, void *o, void *od, float *lse, float *lse_dot, int B, int H, int Lq,
                   int Lk, int d, float scale, const int32_t *kv_len, void *stream, uint64_t timeout_ns,
                   int flags, bool allow_zero_kv, unsigned long long *trace = nullptr, int trace_tiles = 0,
-                  int trace_ctas = 0)
+                  int trace_ctas = 0, void *workspace = nullptr, size_t workspace_bytes = 0,
+                  bool use_split = false)
 {
     const bool zkv = allow_zero_kv && !kd && !vd;
     if (!q || !k || !v || !qd || (!zkv && (!kd || !vd)) || !o || !od || !lse) return ATTN_JVP_ERR_NULL;
@@ -1309,6 +1557,25 @@ static int launch(const void *q, const void *k, const void *v, const void *qd, c
 
     const int nqt = (Lq + BM - 1) / BM;
     const long long n_tiles = static_cast<long long>(nqt) * BH;  // < 2^31 / BM by the check above
+    int n_sm = 0;
+    if (int rc = device_sms(&n_sm)) return rc;
+    SplitPlan sp;
+    if (use_split) {
+        sp = split_plan(n_tiles, n_sm, Lk, d);
+    } else {  // every tile whole, round robin over min(tiles, SMs) CTAs
+        sp.grid = static_cast<int>(n_tiles < n_sm ? n_tiles : n_sm);
+        sp.n_full = static_cast<int>(n_tiles);
+    }
+    const size_t nws = use_split ? sp.bytes : 0;
+    if (nws) {
+        if (!workspace) return ATTN_JVP_ERR_NULL;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255) return ATTN_JVP_ERR_ALIGN;
+        if (workspace_bytes < nws) return ATTN_JVP_ERR_VALUE;
+        for (int j = 0; j < 6; ++j)
+            if (ins[j] && ranges_overlap(workspace, nws, ins[j], insz[j])) return ATTN_JVP_ERR_VALUE;
+        for (int j = 0; j < 5; ++j)
+            if (outs[j] && ranges_overlap(workspace, nws, outs[j], outsz[j])) return ATTN_JVP_ERR_VALUE;
+    }
 
     Params prm;
     std::memset(&prm, 0, sizeof prm);
@@ -1334,12 +1601,21 @@ static int launch(const void *q, const void *k, const void *v, const void *qd, c
     prm.trace = trace;
     prm.trace_tiles = trace_tiles;
     prm.trace_ctas = trace_ctas;
-
+    prm.n_full = sp.n_full;
+    prm.split_S = sp.S;
+    prm.n_units = sp.n_units;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (nws) {
+        prm.cnt = static_cast<int *>(workspace);
+        prm.part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + sp.cnt_bytes);
+        if (cudaMemsetAsync(workspace, 0, sp.cnt_bytes, s) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
+    }
+
     int rc;
-    if (trace) rc = d == 64 ? launch_kernel<64, false, true>(prm, s) : launch_kernel<128, false, true>(prm, s);
-    else if (zkv) rc = d == 64 ? launch_kernel<64, true>(prm, s) : launch_kernel<128, true>(prm, s);
-    else rc = d == 64 ? launch_kernel<64, false>(prm, s) : launch_kernel<128, false>(prm, s);
+    const int grid = sp.grid;
+    if (trace) rc = d == 64 ? launch_kernel<64, false, true>(prm, grid, s) : launch_kernel<128, false, true>(prm, grid, s);
+    else if (zkv) rc = d == 64 ? launch_kernel<64, true>(prm, grid, s) : launch_kernel<128, true>(prm, grid, s);
+    else rc = d == 64 ? launch_kernel<64, false>(prm, grid, s) : launch_kernel<128, false>(prm, grid, s);
     if (rc) return rc;
     if (cudaGetLastError() != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     return ATTN_JVP_OK;
@@ -1365,6 +1641,26 @@ int attn_jvp_fwd_ex(const void *q, const void *k, const void *v, const void *q_d
                         kv_len, stream, 0, 0, true);
 }
 
+size_t attn_jvp_workspace_bytes(int B, int H, int Lq, int Lk, int d)
+{
+    if (B < 1 || H < 1 || Lq < 1 || Lk < 1 || (d != 64 && d != 128)) return 0;
+    const long long BH = static_cast<long long>(B) * H;
+    if (BH * Lq >= (1ll << 31) || BH * Lk >= (1ll << 31)) return 0;
+    int n_sm = 0;
+    if (ajvp::device_sms(&n_sm)) return 0;
+    const long long T = static_cast<long long>((Lq + ajvp::BM - 1) / ajvp::BM) * BH;
+    return ajvp::split_plan(T, n_sm, Lk, d).bytes;
+}
+
+int attn_jvp_fwd_ws(const void *q, const void *k, const void *v, const void *q_dot, const void *k_dot,
+                    const void *v_dot, void *o, void *o_dot, float *lse, float *lse_dot, int B, int H,
+                    int Lq, int Lk, int d, float scale, const int32_t *kv_len, void *workspace,
+                    size_t workspace_bytes, void *stream)
+{
+    return ajvp::launch(q, k, v, q_dot, k_dot, v_dot, o, o_dot, lse, lse_dot, B, H, Lq, Lk, d, scale,
+                        kv_len, stream, 0, 0, true, nullptr, 0, 0, workspace, workspace_bytes, true);
+}
+
 int attn_jvp_fwd_debug(const void *q, const void *k, const void *v, const void *q_dot,
                        const void *k_dot, const void *v_dot, void *o, void *o_dot, float *lse, int B,
                        int H, int Lq, int Lk, int d, float scale, const int32_t *kv_len, void *stream,
@@ -1387,13 +1683,15 @@ int attn_jvp_fwd_trace(const void *q, const void *k, const void *v, const void *
 int attn_jvp_check(void *stream, int *site)
 {
     if (site) *site = 0;
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return ATTN_JVP_ERR_LAUNCH;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(ajvp::g_check_mu);
+    ajvp::take_status_kernel<<<1, 1, 0, s>>>();
+    if (cudaGetLastError() != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     int st = 0;
-    if (cudaMemcpyFromSymbol(&st, ajvp::g_status, sizeof st) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
+    if (cudaMemcpyFromSymbolAsync(&st, ajvp::g_status_taken, sizeof st, 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return ATTN_JVP_ERR_LAUNCH;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     if (st == 0) return ATTN_JVP_OK;
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(ajvp::g_status, &zero, sizeof zero) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     if (site) *site = st;
     return ATTN_JVP_ERR_TIMEOUT;
 }

@@ -79,6 +79,15 @@ struct Params {
 };
 
 __device__ int g_status;
+__device__ int g_status_taken;  // the word as the last check took it
+
+// Read and clear the status word in one atomic step, ordered on the checking
+// stream, so a site recorded by a kernel on another stream between a read
+// and a clear cannot be lost.
+__global__ void take_status_kernel() { g_status_taken = atomicExch(&g_status, 0); }
+
+// Host threads that check at the same time take turns on g_status_taken.
+static std::mutex g_check_mu;
 
 // Bounded wait (acquire at cluster scope: most of these barriers are
 // signalled from the other CTA of the pair); gives up when another role has
@@ -500,12 +509,15 @@ int qkv_rmsnorm_jvp(const void *x, const void *x_dot, const void *w_qkv, const f
 int qkv_prologue_check(void *stream, int *site)
 {
     if (site) *site = 0;
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(qkvp::g_check_mu);
+    qkvp::take_status_kernel<<<1, 1, 0, s>>>();
+    if (cudaGetLastError() != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     int st = 0;
-    if (cudaMemcpyFromSymbol(&st, qkvp::g_status, sizeof st) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
+    if (cudaMemcpyFromSymbolAsync(&st, qkvp::g_status_taken, sizeof st, 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return ATTN_JVP_ERR_LAUNCH;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     if (st == 0) return ATTN_JVP_OK;
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(qkvp::g_status, &zero, sizeof zero) != cudaSuccess) return ATTN_JVP_ERR_LAUNCH;
     if (site) *site = st;
     return ATTN_JVP_ERR_TIMEOUT;
 }

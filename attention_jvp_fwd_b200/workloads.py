@@ -196,6 +196,9 @@ NAMED = {
     "cross_frozen": dict(B=4, H=16, Lq=4096, Lk=512, d=128),
     # T2V self-attention, 21 latent frames x 30 x 52 patches (14B-DiT-like)
     "t2v_self": dict(B=1, H=40, Lq=32760, Lk=32760, d=128),
+    # the same heads at a quarter of the length: small enough for profiler
+    # captures, with the same per-head layout and recipe
+    "t2v_self_L8192": dict(B=1, H=40, Lq=8192, Lk=8192, d=128),
 }
 for _n in _stress_names() + _stress_sharp_names():
     _d = int(_n.split("_d")[1].split("_")[0])
@@ -221,7 +224,8 @@ def make(name: str, seed: int = 0) -> Workload:
     - ``cross``: all N(0, 1); kv_len[b] ~ U{64..512}; K' = V' = 0 for the
       second half of the batch (frozen text tokens).
     - ``cross_frozen``: as ``cross`` with K' = V' = 0 for every batch.
-    - ``t2v_self``: Q, K rows at unit RMS; V and tangents N(0, 1).
+    - ``t2v_self``: Q, K rows at unit RMS; V and tangents N(0, 1);
+      ``t2v_self_L8192`` is the same recipe at L = 8192.
     - ``stress_d{d}_L{L}``: Q x 4; tangents x 10**u, u ~ U[-3, 1] per head.
     - ``stress_sharp_d{d}_L{L}``: as stress but Q x 10, which puts the logit
       standard deviation near 10 and the extremes near +-60.
@@ -238,7 +242,7 @@ def make(name: str, seed: int = 0) -> Workload:
         kv = rng.integers(64, 513, size=B).astype(np.int32)
         return make_custom(B, H, Lq, Lk, d, seed, name=name, kv_len=kv,
                            zero_kv_dot_from=B // 2 if name == "cross" else 0)
-    if name == "t2v_self":
+    if name in ("t2v_self", "t2v_self_L8192"):
         return make_custom(B, H, Lq, Lk, d, seed, name=name, unit_rms_qk=True)
     if name.startswith("stress_sharp_"):
         return make_custom(B, H, Lq, Lk, d, seed, name=name, q_gain=10.0,

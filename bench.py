@@ -2,8 +2,8 @@
 """Benchmark of the fused attention forward + JVP on B200.
 
 One step = one call of the whole path (one kernel launch) over one batch of a
-named synthetic workload (default: T2I self-attention, B=2 H=16 L=4096
-d=128).  Prints ONE JSON line on rank 0.
+named synthetic workload (default: T2V self-attention, B=1 H=40 L=32760
+d=128, the largest single-GPU configuration).  Prints ONE JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl ours|reference] [--no-cpu-baseline]
@@ -15,6 +15,10 @@ FLOPs / the slowest rank's time.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded
 row sample of the same workload (rank 0 only).
+
+The roofline object names the bound from the workload's arithmetic intensity
+(FLOPs performed over algorithmic bytes) against the ridge point of the two
+measured peaks, and carries both the tensor and the HBM fraction.
 """
 from __future__ import annotations
 
@@ -26,6 +30,7 @@ import math
 import os
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -50,16 +55,25 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: about 10 s of kernel time for the workload)")
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="t2i_self")
+    ap.add_argument("--workload", default="t2v_self")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--e2e-steps", type=int, default=0, help="0 = min(steps, 100)")
-    return ap.parse_args(argv)
+    args = ap.parse_args(argv)
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS.get(args.workload, 1000)
+    return args
+
+
+# default timed steps per workload: about 10 s of kernel time (T2V is 54 ms
+# a launch), 1000 launches elsewhere
+DEFAULT_STEPS = {"t2v_self": 200}
 
 
 # ----------------------------------------------------------------- helpers
@@ -122,18 +136,19 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu_index = gpu_index
+    def __init__(self, device):
+        # nvidia-smi numbers GPUs without regard to CUDA_VISIBLE_DEVICES, so
+        # the device is named by its UUID (else its PCI bus id)
+        self.gpu_id = smi_device_id(device)
         self.proc = None
         self.path = None
 
     def start(self):
         try:
-            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{self.gpu_index}.csv")
-            self.f = open(self.path, "w")
+            fd, self.path = tempfile.mkstemp(prefix="bench_clocks_", suffix=".csv")
+            self.f = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
         except OSError:
@@ -150,17 +165,22 @@ class ClockSampler:
         self.f.close()
         rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 10:
-                    continue
-                try:
-                    rows.append({"sm": float(parts[2]), "max": float(parts[3]),
-                                 "power": float(parts[4]),
-                                 "hw": parts[6], "hw_th": parts[7], "sw_th": parts[8],
-                                 "sw_pc": parts[9]})
-                except ValueError:
-                    continue
+            lines = f.readlines()
+        try:
+            os.unlink(self.path)
+        except OSError:
+            pass
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append({"sm": float(parts[2]), "max": float(parts[3]),
+                             "power": float(parts[4]),
+                             "hw": parts[6], "hw_th": parts[7], "sw_th": parts[8],
+                             "sw_pc": parts[9]})
+            except ValueError:
+                continue
         if not rows:
             return None
         load = [r for r in rows if r["power"] > 200.0] or rows
@@ -172,7 +192,27 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": float(np.median([r["sm"] for r in load])),
                 "sm_max_mhz": float(max(r["max"] for r in rows)),
-                "reasons": sorted(reasons), "samples": len(load)}
+                "reasons": sorted(reasons), "samples": len(load), "gpu": self.gpu_id}
+
+
+def smi_device_id(device) -> str:
+    """The nvidia-smi --id of a torch CUDA device: 'GPU-<uuid>', else the PCI
+    bus id, else the CUDA ordinal."""
+    import torch
+    props = torch.cuda.get_device_properties(device)
+    uuid = str(getattr(props, "uuid", "") or "")
+    if uuid:
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    if hasattr(props, "pci_bus_id"):
+        return "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+    return str(torch.device(device).index or 0)
+
+
+def roofline_bound(flops: float, nbytes: float, peak_tf: float, peak_hbm_gbs: float) -> str:
+    """'tensor' when the arithmetic intensity (FLOP per algorithmic byte) is
+    above the ridge point of the two peaks, else 'hbm'."""
+    ridge = peak_tf * 1e12 / (peak_hbm_gbs * 1e9)
+    return "tensor" if flops / nbytes > ridge else "hbm"
 
 
 # ----------------------------------------------------------------- distributed
@@ -252,24 +292,41 @@ def stream_e2e(dev, host_ins, out_like, call, steps, group):
 
 # ----------------------------------------------------------------- CPU oracle
 
+# The oracle runs the whole workload when a probe says that takes at most
+# this long; otherwise it runs a row sample and its rate stands for the rest.
+FULL_ORACLE_S = 60.0
+
+
 def time_oracle(w, seconds: float, seed: int = 123):
-    """Time the fp64 oracle on a row sample sized for about `seconds`."""
+    """Time the fp64 oracle: the whole workload if the probe's estimate is at
+    most FULL_ORACLE_S, else a random row sample sized for about `seconds`.
+    Returns (TFLOP/s, cores, rows run, seconds, sample description)."""
     import oracle
     rng = np.random.default_rng(seed)
     total_rows = w.B * w.H * w.Lq
     cores = oracle.max_threads()
-    probe = min(total_rows, max(cores * 2, 16))
+    probe = min(total_rows, max(cores * 4, 64))
     rows = np.sort(rng.choice(total_rows, size=probe, replace=False)).astype(np.int64)
     t0 = time.perf_counter()
     oracle.attn_jvp(*w.inputs(), w.scale, kv_len=w.kv_len, rows=rows)
     dt = max(time.perf_counter() - t0, 1e-6)
+    est_full = dt * total_rows / probe
+    if est_full <= FULL_ORACLE_S:
+        t0 = time.perf_counter()
+        oracle.attn_jvp(*w.inputs(), w.scale, kv_len=w.kv_len)
+        dt = time.perf_counter() - t0
+        v = w.flops_valid() / dt / 1e12
+        return v, cores, total_rows, dt, f"full run of {w.name} ({total_rows} query rows), {dt:.1f} s"
     n = int(min(total_rows, max(probe, probe * seconds / dt)))
     rows = np.sort(rng.choice(total_rows, size=n, replace=False)).astype(np.int64)
     t0 = time.perf_counter()
     oracle.attn_jvp(*w.inputs(), w.scale, kv_len=w.kv_len, rows=rows)
     dt = time.perf_counter() - t0
-    flops = row_flops(w, rows)
-    return flops / dt / 1e12, cores, n, dt
+    v = row_flops(w, rows) / dt / 1e12
+    full_s = w.flops_valid() / (v * 1e12)
+    return v, cores, n, dt, (f"{n} random query rows of {w.name} (of {total_rows}, all keys of each), "
+                             f"{dt:.1f} s; a full run would take about {full_s:.0f} s at this rate "
+                             f"(extrapolated, not run)")
 
 
 def row_flops(w, rows) -> float:
@@ -387,7 +444,7 @@ def run_ours(args):
     if st != 0:
         raise RuntimeError(f"device status {st} at site {site} after warm-up")
 
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(dev)
     sampler.start()
     time.sleep(0.6)
     if group:
@@ -449,19 +506,28 @@ def run_ours(args):
     # the roofline counts what the kernel performs: 8 units with K' = V' = 0
     achieved = w.flops_performed() / (per_launch_ms * 1e-3) / 1e12
     traffic = measured_traffic(args.workload)
+    alg_bytes = algorithmic_bytes(w)
+    achieved_gbs = alg_bytes / (per_launch_ms * 1e-3) / 1e9
+    bound = roofline_bound(w.flops_performed(), alg_bytes, peak_tf, peak_hbm)
+    tensor_side = {"achieved": achieved, "peak": peak_tf, "unit": UNIT, "frac": achieved / peak_tf,
+                   "frac_of_burst_peak": achieved / burst_tf,
+                   "peak_source": f"{peak_src} bf16 dense ({peak_kind}; timed region {local_ms:.0f} ms)"}
+    hbm_side = {"achieved": achieved_gbs, "peak": peak_hbm, "unit": "GB/s",
+                "frac": achieved_gbs / peak_hbm, "peak_source": f"{peak_src} HBM copy bandwidth"}
+    main_side, other_side = (tensor_side, hbm_side) if bound == "tensor" else (hbm_side, tensor_side)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(w, args),
         "gpu_launches": args.steps,
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf,
-                     "peak_source": f"{peak_src} bf16 dense ({peak_kind}; timed region "
-                                    f"{local_ms:.0f} ms)", "unit": UNIT,
-                     "frac": achieved / peak_tf, "frac_of_burst_peak": achieved / burst_tf,
+        "roofline": {"bound": bound, **main_side,
                      "traffic": traffic,
-                     "algorithmic_bytes": algorithmic_bytes(w),
+                     "algorithmic_bytes": alg_bytes,
                      "flops_per_launch": w.flops_performed(),
+                     "intensity_flop_per_byte": w.flops_performed() / alg_bytes,
+                     "ridge_flop_per_byte": peak_tf * 1e12 / (peak_hbm * 1e9),
+                     "tensor" if bound == "hbm" else "hbm": other_side,
                      "kernel": f"attn_jvp_fwd_kernel<{d}>"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "how": E2E_NOTE},
@@ -475,10 +541,9 @@ def run_ours(args):
                                   "the 12 FLOP units; value counts the metric's 12 units, "
                                   "roofline.achieved the 8 performed")
     if rank == 0 and not group and not args.no_cpu_baseline:
-        v, cores, n, dt = time_oracle(w, args.cpu_seconds)
+        v, cores, n, dt, sample = time_oracle(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"{n} random query rows of {w.name} (all keys), "
-                                          f"{dt:.1f} s"}
+                                "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if group:
@@ -539,7 +604,7 @@ def run_loss(args):
         for _ in range(args.warmup):
             step()
     torch.cuda.synchronize(dev)
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(dev)
     sampler.start()
     time.sleep(0.6)
     if group:
@@ -743,7 +808,7 @@ def run_qkv(args):
     st, site = A.qkv_prologue_check(stream)
     if st != 0:
         raise RuntimeError(f"device status {st} at site {site}")
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(dev)
     sampler.start()
     time.sleep(0.6)
     if group:

@@ -44,6 +44,7 @@
 #ifndef ATTN_JVP_H
 #define ATTN_JVP_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -116,12 +117,61 @@ int attn_jvp_fwd_ex(const void *q, const void *k, const void *v,
                     const int32_t *kv_len, void *stream);
 
 /*
- * attn_jvp_check -- synchronise `stream`, then read and clear the current
- * device's status word.  Returns ATTN_JVP_OK, ATTN_JVP_ERR_TIMEOUT if a
- * kernel launched since the last check gave up on a pipeline wait (its
- * outputs are then unspecified), or ATTN_JVP_ERR_LAUNCH if the
- * synchronisation itself failed.  If `site` is not NULL it receives the code
- * of the first wait that gave up (0 if none).
+ * attn_jvp_fwd_ws -- attn_jvp_fwd_ex with the last wave of query tiles split
+ * over the key range.  The kernel keeps one persistent CTA per SM; with T
+ * query tiles ([ceil(Lq / 128)] * B * H) on n SMs, the last T mod n tiles
+ * would leave most SMs idle for a whole tile's time.  Each of them is cut
+ * instead into S = min(n / (T mod n), ceil(Lk / 64), 8) key ranges, one per
+ * CTA.  Every range keeps the unnormalised online-softmax state of its keys
+ * (running max m, l = sum p, a = sum p (s S' - c), the centring constant c,
+ * O_acc and O'_acc) and writes it to `workspace`; the range that finishes
+ * last merges the states of its tile (the same rescaling by 2^(m - max m)
+ * that the online softmax applies between key tiles) and writes the
+ * outputs.  No CTA waits for another.  The results equal attn_jvp_fwd_ex's
+ * up to the order of the fp32 sums.  This is the FlashAttention-2 forward's
+ * block-wise online softmax (rCM pages: ai.info AI summary, Key
+ * Contributions 1 and Methodology in Plain English; papernotes.org notes,
+ * key design 1), with blocks of keys taken by different CTAs; the pages do
+ * not describe a split.
+ *   workspace        device memory of at least attn_jvp_workspace_bytes(B, H,
+ *                    Lq, Lk, d) bytes, 256-byte aligned, not overlapping any
+ *                    other argument; caller-owned.  Its first bytes are
+ *                    counters that the call zeroes (cudaMemsetAsync on
+ *                    `stream`) before the kernel; the rest is overwritten.
+ *                    Calls that run at the same time need separate
+ *                    workspaces.  NULL is allowed when the size is 0 (no
+ *                    split for this shape on this device).
+ *   workspace_bytes  its size; less than needed is ATTN_JVP_ERR_VALUE.
+ * Everything else is as for attn_jvp_fwd_ex.
+ */
+int attn_jvp_fwd_ws(const void *q, const void *k, const void *v,
+                    const void *q_dot, const void *k_dot, const void *v_dot,
+                    void *o, void *o_dot, float *lse, float *lse_dot,
+                    int B, int H, int Lq, int Lk, int d, float scale,
+                    const int32_t *kv_len, void *workspace, size_t workspace_bytes,
+                    void *stream);
+
+/*
+ * attn_jvp_workspace_bytes -- bytes of workspace attn_jvp_fwd_ws needs for
+ * this shape on the current device (it depends on the SM count); 0 when the
+ * shape gets no split or the arguments are out of range.  There are at most
+ * n ranges (n SMs), so it is at most 256 + n * (4 + 2 d) * 128 * 4 bytes:
+ * 19.7 MB at d = 128, 10.0 MB at d = 64 on a 148-SM B200.
+ */
+size_t attn_jvp_workspace_bytes(int B, int H, int Lq, int Lk, int d);
+
+/*
+ * attn_jvp_check -- take the current device's status word: a one-thread
+ * kernel queued on `stream` reads and clears it in one atomic exchange, and
+ * the call then synchronises `stream`.  Returns ATTN_JVP_OK,
+ * ATTN_JVP_ERR_TIMEOUT if a kernel that finished before the exchange gave up
+ * on a pipeline wait (its outputs are then unspecified), or
+ * ATTN_JVP_ERR_LAUNCH if the launch or the synchronisation failed.  If `site`
+ * is not NULL it receives the code of the first wait that gave up (0 if none).
+ * The word is per device, not per stream: a check on one stream also reports
+ * (and clears) a timeout of a kernel on another stream of the same device,
+ * if that kernel finished before the exchange ran.  Host threads that check
+ * at the same time take turns; no recorded site is lost.
  */
 int attn_jvp_check(void *stream, int *site);
 

@@ -157,3 +157,27 @@ def test_outputs_16_byte_aligned(d):
     ref = [t.clone() for t in attn_jvp_fwd(*ins, scale=w.scale)]
     torch.cuda.synchronize()
     assert torch.equal(o, ref[0]) and torch.equal(od, ref[1]) and torch.equal(lse, ref[2])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("masked", [False, True])
+def test_centring_window_underflow(d, masked):
+    """One dominant key at index 40 and keys 0..31 about 120 logits below it:
+    in the first key tile every p of keys 0..31 underflows to exactly 0, so
+    the p-weighted centring window has zero weight.  The outputs must stay
+    finite and match the oracle (the centring constant cancels in exact
+    arithmetic, so the kernel may take any finite value there)."""
+    B, H, Lq, Lk = 2, 2, 130, 200
+    w = W.make_custom(B, H, Lq, Lk, d, seed=41,
+                      kv_len=np.array([41, 200], np.int32) if masked else None)
+    q = 0.1 * W.bf16_bits_to_f32(w.q)
+    k = 0.1 * W.bf16_bits_to_f32(w.k)
+    q[..., 0] = 10.0
+    k[..., :32, 0] = -10.0   # keys 0..31: logit about -100 at scale 1
+    k[..., 40, 0] = 2.0      # key 40: about +20
+    w.q = W.bf16_round_bits(q)
+    w.k = W.bf16_round_bits(k)
+    o, od, lse = run_gpu(w, scale=1.0)
+    assert bool(torch.all(torch.isfinite(o.float()))) and bool(torch.all(torch.isfinite(od.float())))
+    assert bool(torch.all(torch.isfinite(lse)))
+    compare(gpu_rows(o, od, lse), oracle_ref(w, scale=1.0), f"centring underflow d{d} masked={masked}")

@@ -41,3 +41,24 @@ def test_single_rank_ulysses_is_the_kernel(nccl_group):
     torch.cuda.synchronize()
     assert torch.equal(o, ro) and torch.equal(od, rod) and torch.equal(lse, rlse)
     compare(gpu_rows(o, od, lse), oracle_ref(w), "ulysses P=1")
+
+
+@pytest.mark.parametrize("zero_kv", [False, True])
+def test_single_rank_ulysses_cross(nccl_group, zero_kv):
+    """Cross-attention through the context-parallel call: text keys replicated
+    (Lk = 77, ragged valid lengths including 0), with and without K' = V' = 0,
+    with the lse tangent.  At P = 1 it must be the plain kernel call, bit for
+    bit, and match the oracle."""
+    kv = np.array([77, 0, 30], np.int32)
+    w = W.make_custom(3, 4, 260, 77, 128, seed=43, kv_len=kv,
+                      zero_kv_dot_from=0 if zero_kv else None)
+    ins = [to_dev(x) for x in w.inputs()]
+    if zero_kv:
+        ins[4] = ins[5] = None
+    kvt = torch.from_numpy(kv).cuda()
+    got = ulysses.ulysses_attn_jvp(*ins, scale=w.scale, kv_len=kvt, lse_dot=True, kv_layout="replicated")
+    ref = attn_jvp_fwd(*ins, scale=w.scale, kv_len=kvt, lse_dot=True)
+    torch.cuda.synchronize()
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
+    compare(gpu_rows(*got[:3]), oracle_ref(w), f"ulysses cross P=1 zero_kv={zero_kv}")
