@@ -11,8 +11,9 @@ layer that produces attention's inputs and their tangents.
 from .api import (ATTN_JVP_ERR_ALIGN, ATTN_JVP_ERR_HEADDIM, ATTN_JVP_ERR_LAUNCH,  # noqa: F401
                   ATTN_JVP_ERR_NULL, ATTN_JVP_ERR_SHAPE, ATTN_JVP_ERR_TIMEOUT,
                   ATTN_JVP_ERR_VALUE, ATTN_JVP_OK, AttnJvpError, attn_jvp_check,
-                  attn_jvp_fwd, attn_jvp_fwd_trace, attn_jvp_status_string, library_path,
+                  attn_jvp_fwd, attn_jvp_fwd_trace, attn_jvp_status_string, attn_jvp_workspace_bytes,
+                  library_path,
                   qkv_prologue_check, qkv_rmsnorm_jvp, scm_tangent_loss)
 
-__all__ = ["attn_jvp_fwd", "attn_jvp_fwd_trace", "attn_jvp_check", "attn_jvp_status_string",
+__all__ = ["attn_jvp_fwd", "attn_jvp_fwd_trace", "attn_jvp_workspace_bytes", "attn_jvp_check", "attn_jvp_status_string",
            "AttnJvpError", "library_path", "scm_tangent_loss", "qkv_rmsnorm_jvp", "qkv_prologue_check"]

@@ -138,6 +138,12 @@ struct Cfg {
     static constexpr uint32_t IDESC_PVV = idesc_bf16_f32(BM, 2 * D, true);
     static_assert(2 * D <= 256, "one MMA covers at most 256 columns");
     static constexpr int P_ARRIVALS = ALT ? 4 : 8;  // one per softmax warp that writes the tile
+    // quarters of the softmax's exponentials computed on the FMA pipe
+    // (ex2_poly2); the rest go to the MUFU unit.  Measured (alternating
+    // timing, same inputs): at d = 128 one quarter is 1.9 % faster on T2I
+    // than none, two are even, three are 2.5 % slower; at d = 64 every
+    // fraction is slower (1.5 % at one quarter), so none is used there.
+    static constexpr int POLY_QUARTERS = D == 64 ? 0 : 1;
     static_assert(T_S + 4 * BN <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -334,6 +340,35 @@ __device__ __forceinline__ bool wait_bar_fast(uint64_t *bar, uint32_t parity, co
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 __device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
 
+// 2^a, 2^b (a, b below 2^7) on the FMA pipe, so that the softmax's exponentials
+// are shared between the MUFU unit (ex2.approx) and the FMA units instead of
+// queueing on the MUFU alone.  Cody-Waite range reduction: t = j + f with j
+// the nearest integer (t + 1.5 * 2^23 rounds it into the low mantissa bits)
+// and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients
+// were fitted here for relative error (at most 7.5e-5 in fp32 Horner form,
+// well below the 2^-9 rounding of the bf16 P it feeds); j is then added to
+// the exponent field.  Arguments below -125 are raised to -125 (a result
+// near 2^-125, where ex2.approx.ftz would give 0; both are negligible
+// against the row sum, which holds a term of at least 1/16).
+__device__ __forceinline__ void ex2_poly2(float a, float b, float &ya, float &yb)
+{
+    constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23
+    const uint64_t t = f2_pack(fmaxf(a, -125.0f), fmaxf(b, -125.0f));
+    const uint64_t r = f2_add(t, f2_pack(MAGIC, MAGIC));
+    const uint64_t j = f2_add(r, f2_pack(-MAGIC, -MAGIC));
+    const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), t);  // t - j, exact
+    uint64_t q = f2_fma(f, f2_pack(0.05517115443944931f, 0.05517115443944931f),
+                        f2_pack(0.2426101416349411f, 0.2426101416349411f));
+    q = f2_fma(q, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+    q = f2_fma(q, f, f2_pack(0.9999281167984009f, 0.9999281167984009f));
+    float qa, qb, ra, rb;
+    f2_unpack(q, qa, qb);
+    f2_unpack(r, ra, rb);
+    // the low bits of r hold 0x4B400000 + j: shifted by 23 they add j to q's exponent
+    ya = __uint_as_float(f2u(ra) * 8388608u + f2u(qa));
+    yb = __uint_as_float(f2u(rb) * 8388608u + f2u(qb));
+}
+
 // Max (or min) of the 64 floats held as bits in a and b, as a balanced tree
 // of 3-input operations (32 of them).  Exact, so the order of the two halves
 // does not change the result.
@@ -397,7 +432,7 @@ __device__ __forceinline__ void part_put_cols(const Params &p, int u, int r, int
 // and writes the outputs (warpgroup 0: O and lse, warpgroup 1: O' and lse').
 // No CTA waits for another: the ranges that finish earlier just leave.
 template <int D>
-__device__ __noinline__ void split_finish(const Params &p, const Tile &t, int g, int r, int lane, __nv_bfloat16 *out_ptr,
+__device__ __noinline__ void split_finish(const Params &p, const Tile &t, int g, int r, __nv_bfloat16 *out_ptr,
                              int grow, size_t lrow, uint8_t *flag_smem)
 {
     volatile int *flag = reinterpret_cast<volatile int *>(flag_smem);
@@ -439,10 +474,16 @@ __device__ __noinline__ void split_finish(const Params &p, const Tile &t, int g,
                 for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, __ldcg(od + i * BM), fmaf(kk, __ldcg(o + i * BM), acc[i]));
             }
         }
-        uint32_t pv[16];
+        // 16-byte stores of the thread's own row (the merge runs for a few
+        // tiles only, so the paired 32-byte stores of the main epilogue buy
+        // nothing here)
+        if (grow < p.Lq) {
+            uint4 *d4 = reinterpret_cast<uint4 *>(out_ptr + c);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
-        store_cols32<D>(out_ptr, c, pv, p.out_v8, lane & 1, (grow & ~1) < p.Lq, (grow | 1) < p.Lq);
+            for (int i = 0; i < 4; ++i)
+                d4[i] = make_uint4(pack_bf16x2(acc[8 * i], acc[8 * i + 1]), pack_bf16x2(acc[8 * i + 2], acc[8 * i + 3]),
+                                   pack_bf16x2(acc[8 * i + 4], acc[8 * i + 5]), pack_bf16x2(acc[8 * i + 6], acc[8 * i + 7]));
+        }
     }
     if (g == 0 && grow < p.Lq) p.lse[lrow] = (M + log2f(L)) * 0.69314718055994531f;
     if (g == 1 && p.lse_dot && grow < p.Lq) p.lse_dot[lrow] = mu;
@@ -848,10 +889,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                             float t0, t1, t2, t3;
                             f2_unpack(f2_fma(f2_pack(u2f(ra[2 * i]), u2f(ra[2 * i + 1])), sl22, nm2), t0, t1);
                             f2_unpack(f2_fma(f2_pack(u2f(rb[2 * i]), u2f(rb[2 * i + 1])), sl22, nm2), t2, t3);
-                            x[2 * i] = ex2_approx(t0);
-                            x[2 * i + 1] = ex2_approx(t1);
-                            x[32 + 2 * i] = ex2_approx(t2);
-                            x[33 + 2 * i] = ex2_approx(t3);
+                            // pairs (i, a) and (i, b): quarter q of the 4 values goes to the
+                            // FMA pipe when q < POLY_QUARTERS (b pairs first, odd i first)
+                            constexpr int PQ = C::POLY_QUARTERS;
+                            const bool poly_b = PQ >= 2 || (PQ == 1 && (i & 1));
+                            const bool poly_a = PQ >= 4 || (PQ == 3 && (i & 1));
+                            if (poly_a) {
+                                ex2_poly2(t0, t1, x[2 * i], x[2 * i + 1]);
+                            } else {
+                                x[2 * i] = ex2_approx(t0);
+                                x[2 * i + 1] = ex2_approx(t1);
+                            }
+                            if (poly_b) {
+                                ex2_poly2(t2, t3, x[32 + 2 * i], x[33 + 2 * i]);
+                            } else {
+                                x[32 + 2 * i] = ex2_approx(t2);
+                                x[33 + 2 * i] = ex2_approx(t3);
+                            }
                         }
                     }
                     if (tail) {
@@ -1061,7 +1115,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     store_cols32<D>(out_ptr, c, pv, p.out_v8, lane & 1, (grow & ~1) < p.Lq, (grow | 1) < p.Lq);
                 }
                 if (part) {
-                    split_finish<D>(p, t, g, r, lane, out_ptr, grow, lrow, smem + C::OFF_MISC + 8);
+                    split_finish<D>(p, t, g, r, out_ptr, grow, lrow, smem + C::OFF_MISC + 8);
                 } else {
                     if (g == 0 && grow < p.Lq) p.lse[lrow] = (M + log2f(lt)) * 0.69314718055994531f;
                     if (g == 1 && p.lse_dot && grow < p.Lq) p.lse_dot[lrow] = mu;
@@ -1167,8 +1221,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     for (int i = 0; i < 16; ++i) {
                         float t0, t1;
                         f2_unpack(f2_fma(f2_pack(u2f(ra[2 * i]), u2f(ra[2 * i + 1])), sl22, nm2), t0, t1);
-                        x[2 * i] = ex2_approx(t0);
-                        x[2 * i + 1] = ex2_approx(t1);
+                        // pair i goes to the FMA pipe when (i mod 4) < POLY_QUARTERS
+                        if ((i & 3) < C::POLY_QUARTERS) {
+                            ex2_poly2(t0, t1, x[2 * i], x[2 * i + 1]);
+                        } else {
+                            x[2 * i] = ex2_approx(t0);
+                            x[2 * i + 1] = ex2_approx(t1);
+                        }
                     }
                 }
                 if (tail) {
@@ -1342,7 +1401,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     for (int i = 0; i < 32; ++i) acc[i] = u2f(v[i]);
                     part_put_cols<D>(p, t.part, r, g, c, acc);
                 }
-                split_finish<D>(p, t, g, r, lane, out_ptr, grow, lrow, smem + C::OFF_MISC + 8);
+                split_finish<D>(p, t, g, r, out_ptr, grow, lrow, smem + C::OFF_MISC + 8);
                 continue;
             }
 #pragma unroll 1
