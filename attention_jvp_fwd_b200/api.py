@@ -23,9 +23,11 @@ ATTN_JVP_ERR_ALIGN = -4
 ATTN_JVP_ERR_LAUNCH = -5
 ATTN_JVP_ERR_TIMEOUT = -6
 ATTN_JVP_ERR_VALUE = -7
+ATTN_JVP_ERR_SCRATCH = -8
 ATTN_JVP_DEBUG_STARVE_Q = 1
 
 EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_ex", "attn_jvp_fwd_ws", "attn_jvp_workspace_bytes",
+            "attn_jvp_fwd_noalloc",
             "attn_jvp_fwd_debug", "attn_jvp_fwd_trace", "attn_jvp_check", "attn_jvp_status_string", "attn_jvp_version", "scm_tangent_loss",
             "qkv_rmsnorm_jvp", "qkv_prologue_check")
 TRACE_EVENTS = 11  # stamps per key tile of attn_jvp_fwd_trace
@@ -68,6 +70,8 @@ def load_library():
             lib.attn_jvp_fwd_ex.argtypes = [vp] * 10 + [i32] * 5 + [f32, vp, vp]
             lib.attn_jvp_fwd_ws.restype = i32
             lib.attn_jvp_fwd_ws.argtypes = [vp] * 10 + [i32] * 5 + [f32, vp, vp, ctypes.c_size_t, vp]
+            lib.attn_jvp_fwd_noalloc.restype = i32
+            lib.attn_jvp_fwd_noalloc.argtypes = [vp] * 10 + [i32] * 5 + [f32, vp, vp]
             lib.attn_jvp_workspace_bytes.restype = ctypes.c_size_t
             lib.attn_jvp_workspace_bytes.argtypes = [i32] * 5
             lib.attn_jvp_fwd_debug.restype = i32

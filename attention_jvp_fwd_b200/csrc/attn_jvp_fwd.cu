@@ -1680,6 +1680,37 @@ static int launch(const void *q, const void *k, const void *v, const void *qd, c
     return ATTN_JVP_OK;
 }
 
+// ---- the split path with library-owned scratch (attn_jvp_fwd_noalloc)
+//
+// For callers that cannot allocate device memory: runtimes that own all of
+// the device memory and give a kernel library no allocator (only its inputs
+// and outputs), and latency-critical loops that must not call cudaMalloc,
+// which can synchronise the device and stall every stream.  The workspace of
+// the last-wave split lives in this file-scope array instead: every device
+// that loads the library holds its NOALLOC_SCRATCH_BYTES until the process
+// exits, and every call on a device shares it.
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(20) << 20;  // 20 MiB: 148 SMs at d = 128 need 19.7 MB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (host code must not pass the array's name itself: that is a
+// host-side stand-in, not a device address).
+static int noalloc_scratch(void **ptr)
+{
+    static std::mutex mu;
+    static void *addr[MAX_DEVICES] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return ATTN_JVP_ERR_LAUNCH;
+    std::lock_guard<std::mutex> g(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATTN_JVP_ERR_LAUNCH;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return ATTN_JVP_OK;
+}
+
 }  // namespace ajvp
 
 extern "C" {
@@ -1718,6 +1749,28 @@ int attn_jvp_fwd_ws(const void *q, const void *k, const void *v, const void *q_d
 {
     return ajvp::launch(q, k, v, q_dot, k_dot, v_dot, o, o_dot, lse, lse_dot, B, H, Lq, Lk, d, scale,
                         kv_len, stream, 0, 0, true, nullptr, 0, 0, workspace, workspace_bytes, true);
+}
+
+int attn_jvp_fwd_noalloc(const void *q, const void *k, const void *v, const void *q_dot,
+                         const void *k_dot, const void *v_dot, void *o, void *o_dot, float *lse,
+                         float *lse_dot, int B, int H, int Lq, int Lk, int d, float scale,
+                         const int32_t *kv_len, void *stream)
+{
+    // The same checks as attn_jvp_fwd_ws, with the static scratch as the
+    // workspace; a shape whose workspace would not fit is refused before any
+    // CUDA call that touches the scratch.
+    if (B < 1 || H < 1 || Lq < 1 || Lk < 1) return ATTN_JVP_ERR_SHAPE;
+    if (d != 64 && d != 128) return ATTN_JVP_ERR_HEADDIM;
+    const long long BH = static_cast<long long>(B) * H;
+    if (BH * Lq >= (1ll << 31) || BH * Lk >= (1ll << 31)) return ATTN_JVP_ERR_SHAPE;
+    int n_sm = 0;
+    if (int rc = ajvp::device_sms(&n_sm)) return rc;
+    const long long T = static_cast<long long>((Lq + ajvp::BM - 1) / ajvp::BM) * BH;
+    if (ajvp::split_plan(T, n_sm, Lk, d).bytes > ajvp::NOALLOC_SCRATCH_BYTES) return ATTN_JVP_ERR_SCRATCH;
+    void *scratch = nullptr;
+    if (int rc = ajvp::noalloc_scratch(&scratch)) return rc;
+    return ajvp::launch(q, k, v, q_dot, k_dot, v_dot, o, o_dot, lse, lse_dot, B, H, Lq, Lk, d, scale,
+                        kv_len, stream, 0, 0, true, nullptr, 0, 0, scratch, ajvp::NOALLOC_SCRATCH_BYTES, true);
 }
 
 int attn_jvp_fwd_debug(const void *q, const void *k, const void *v, const void *q_dot,
@@ -1766,6 +1819,7 @@ const char *attn_jvp_status_string(int status)
     case ATTN_JVP_ERR_LAUNCH: return "CUDA launch or runtime query failed";
     case ATTN_JVP_ERR_TIMEOUT: return "a device-side pipeline wait gave up";
     case ATTN_JVP_ERR_VALUE: return "scale not finite, or outputs overlap inputs";
+    case ATTN_JVP_ERR_SCRATCH: return "the split workspace this shape needs exceeds the library's static scratch";
     default: return "unknown status";
     }
 }

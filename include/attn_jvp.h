@@ -59,7 +59,9 @@ typedef enum {
     ATTN_JVP_ERR_ALIGN = -4,   /* a tensor pointer is not 16-byte aligned             */
     ATTN_JVP_ERR_LAUNCH = -5,  /* the CUDA runtime refused the launch or a query      */
     ATTN_JVP_ERR_TIMEOUT = -6, /* a device-side wait gave up (see attn_jvp_check)    */
-    ATTN_JVP_ERR_VALUE = -7    /* scale not finite, or outputs overlap inputs         */
+    ATTN_JVP_ERR_VALUE = -7,   /* scale not finite, or outputs overlap inputs         */
+    ATTN_JVP_ERR_SCRATCH = -8  /* attn_jvp_fwd_noalloc: the split needs more than the */
+                               /* library's static scratch holds                      */
 } attn_jvp_status;
 
 /*
@@ -150,6 +152,35 @@ int attn_jvp_fwd_ws(const void *q, const void *k, const void *v,
                     int B, int H, int Lq, int Lk, int d, float scale,
                     const int32_t *kv_len, void *workspace, size_t workspace_bytes,
                     void *stream);
+
+/*
+ * attn_jvp_fwd_noalloc -- attn_jvp_fwd_ws for callers that cannot allocate
+ * device memory: runtimes that own all device memory and give a kernel
+ * library no allocator (only the inputs and outputs), and latency-critical
+ * loops that must not call cudaMalloc, which can synchronise the device and
+ * stall every stream.  The pages have no counterpart: it exists for such
+ * callers.  The caller passes inputs and
+ * outputs exactly as for attn_jvp_fwd_ws, but no workspace: the library uses
+ * a 20 MiB array of its own in device memory, which every GPU that loads the
+ * library holds until the process exits.  The call allocates nothing and
+ * frees nothing.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before
+ *     any stream capture on the device.
+ *   - Every call on a device shares the one array: calls whose kernels can
+ *     overlap on the GPU (different streams without an ordering between
+ *     them) race on it and give wrong results.  The counters in it are
+ *     zeroed on `stream` before each kernel; the rest is overwritten.
+ *   - A shape whose split needs more than the array holds returns
+ *     ATTN_JVP_ERR_SCRATCH (not reachable on a 148-SM B200, where d = 128
+ *     needs at most 19.7 MB).
+ * Everything else is as for attn_jvp_fwd_ws.
+ */
+int attn_jvp_fwd_noalloc(const void *q, const void *k, const void *v,
+                         const void *q_dot, const void *k_dot, const void *v_dot,
+                         void *o, void *o_dot, float *lse, float *lse_dot,
+                         int B, int H, int Lq, int Lk, int d, float scale,
+                         const int32_t *kv_len, void *stream);
 
 /*
  * attn_jvp_workspace_bytes -- bytes of workspace attn_jvp_fwd_ws needs for
