@@ -928,17 +928,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         f2_unpack(f2_add(s1, s3), u2, u3);
                         l += (u0 + u1) + (u2 + u3);
                     }
-                    if (nown >= 1) {
-                        // PV of this warpgroup's previous key tile must be done
-                        // before O_g may be rescaled (it always is by now: its
-                        // o_done phase precedes this tile's S)
-                        if (!__all_sync(0xffffffffu,
-                                        wait_bar_fast(&o_done[g], ((gk >> 1) - 1) & 1, wc, SITE_O_DONE))) {
-                            err = true;
-                            break;
-                        }
-                        tc_fence_after();
-                    }
+                    // The PV MMAs of this warpgroup's previous key tile, which
+                    // write O_g, are done: they were issued before this tile's
+                    // S, and S's commit (seen above) arrives only when every
+                    // MMA issued before it is done.  O_g may be rescaled at once.
                     if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
                         for (int c = 0; c < 2 * D; c += 32) {  // O_g then O'_g
@@ -1238,10 +1231,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-                if (j >= 1) {
-                    // PV of the previous key tile must be done before O may be
-                    // rescaled; a warp cannot fall two phases behind on that V
-                    // slot (the next one needs this warp's P of key tile gk + 1).
+                // The PV MMAs of the previous key tile must be done before O
+                // may be rescaled, so a warp that rescales waits for them.  A
+                // warp that does not rescale skips the wait (most tiles): the
+                // phase it would wait for can never be confused with another,
+                // since S of this tile (seen above) implies that the phases of
+                // key tiles <= gk - 2 are complete, and that of gk + 1 needs
+                // this warp's P of key tile gk + 1.
+                const bool do_rescale = __any_sync(0xffffffffu, rescale);
+                if (j >= 1 && do_rescale) {
                     if (!__all_sync(0xffffffffu, wait_bar_fast(&vo_done[(gk - 1) % C::NV], ((gk - 1) / C::NV) & 1,
                                                                wc, SITE_O_DONE))) {
                         err = true;
@@ -1249,7 +1247,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                     tc_fence_after();
                 }
-                if (__any_sync(0xffffffffu, rescale)) {
+                if (do_rescale) {
                     const uint32_t tacc = tbase + lane_off + (g == 0 ? C::T_O(0) : C::T_OD(0));
 #pragma unroll 1
                     for (int c = 0; c < D; c += 32) {
