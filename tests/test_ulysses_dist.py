@@ -111,7 +111,7 @@ CASES = [
 def test_ulysses_matches_unsharded_oracle(world, case):
     import oracle
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, case, out), nprocs=world, join=True)
         res = dict(out)
