@@ -18,9 +18,10 @@
 //     a = sum p (s S'_raw - c).  At d = 128 each takes one half of every
 //     tile's 64 keys; at d = 64 each takes every other key tile, with its own
 //     m, l, a and accumulators, merged at the end.  They write P and
-//     P (s S'_raw - c) back into TMEM as bf16;
+//     P (s S'_raw - c) as bf16 back into TMEM at d = 128, into shared memory
+//     at d = 64;
 //   * [O | O'_acc] += P [V | V'] (one N = 2d MMA chain) and O'_acc +=
-//     P(sS' - c) V are tcgen05 MMAs with A read from TMEM;
+//     P(sS' - c) V are tcgen05 MMAs with A read from there;
 //   * the epilogue forms O = O_acc / l and O' = (O'_acc - (a / l) O_acc) / l,
 //     while the first S MMAs and loads of the next query tile already run.
 //
@@ -75,6 +76,7 @@ enum : int {
     SITE_DRAIN = 10,
     SITE_SMEM_ALIGN = 11,
     SITE_Q_EMPTY = 12,
+    SITE_S_FREE = 13,
 };
 
 // Two ways to split the softmax between its two warpgroups:
@@ -85,7 +87,10 @@ enum : int {
 //    accumulators O_g, O'_g; the epilogue merges the two.  The two
 //    warpgroups then run out of phase (one's exp2 overlaps the other's
 //    stores), and a row's per-tile latency is spread over two tiles.  The
-//    four accumulators and two S buffers fill TMEM only when d = 64.
+//    four accumulators and two S buffers fill TMEM only when d = 64.  Each
+//    warpgroup has one S buffer, so its P goes to shared memory: the buffer
+//    can then take the warpgroup's next S as soon as S and S'_raw have been
+//    read, while the softmax is still busy with the tile.
 template <int D>
 struct Cfg {
     static constexpr bool ALT = D == 64;
@@ -94,7 +99,8 @@ struct Cfg {
     // and 3 % faster on cross-attention (alternating timing); the 32 KB they
     // leave to the L1 cache is the likely reason.
     static constexpr int NK = (D == 128) ? 2 : 4;
-    static constexpr int NV = (D == 128) ? 2 : 4;    // V ring depth
+    // V ring depth; at d = 64 the P slots take the room of a fourth stage
+    static constexpr int NV = (D == 128) ? 2 : 3;
     static constexpr uint32_t Q_BYTES = BM * D * 2;  // one of Q, Q'
     // K stage: K then K' rows in each column block (one 128-row operand [K; K'])
     static constexpr uint32_t KST_BYTES = 2 * BN * D * 2;
@@ -104,10 +110,18 @@ struct Cfg {
     static constexpr uint32_t OFF_QD = Q_BYTES;
     static constexpr uint32_t OFF_K = 2 * Q_BYTES;
     static constexpr uint32_t OFF_V = OFF_K + NK * KST_BYTES;
-    static constexpr uint32_t OFF_BAR = OFF_V + NV * VST_BYTES;
+    // By tiles the bf16 P and P (sS' - c) operands of the PV MMAs live in
+    // shared memory, one slot of each per warpgroup (128 rows x 64 keys,
+    // K-major with the 128-byte swizzle): the S buffer is then free as soon
+    // as the softmax has read S and S'_raw, and the warpgroup's next S runs
+    // while it still works on this key tile.
+    static constexpr uint32_t P_BYTES = BM * BN * 2;
+    static constexpr uint32_t OFF_P = OFF_V + NV * VST_BYTES;
+    __host__ __device__ static constexpr uint32_t off_p(int g, bool pd) { return OFF_P + (2 * g + (pd ? 1 : 0)) * P_BYTES; }
+    static constexpr uint32_t OFF_BAR = OFF_P + (ALT ? 4 * P_BYTES : 0);
     // q_full, q_empty, k_full[NK], ks_done[NK], v_full[NV], vo_done[NV],
-    // p_full[2], pd_full[2], drain, and by tiles s_full[2], o_done[2]
-    static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 2 + 2 + 1 + (ALT ? 4 : 0);
+    // p_full[2], pd_full[2], drain, and by tiles s_full[2], o_done[2], s_free[2]
+    static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 2 + 2 + 1 + (ALT ? 6 : 0);
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem slot, abort flag
     // Softmax exchange, floats.  By columns: per-warpgroup partial l, a
     // ([2][2][128]) and the centring constant hand-off ([128]).  By tiles:
@@ -122,8 +136,7 @@ struct Cfg {
     // columns and P (sS' - c) over the last 16, so no one overwrites a
     // column another warp may still read.
     //   By tiles the columns are O_0 | O'_0 | O_1 | O'_1 | S buffer 0 | S
-    // buffer 1, and the owner of a buffer writes its bf16 P over S columns
-    // [0, 32) and P (sS' - c) over [32, 64), after it has read all of S.
+    // buffer 1 (warpgroup g's), and P goes to shared memory.
     __host__ __device__ static constexpr uint32_t T_O(int g) { return ALT ? g * 2 * D : 0; }
     __host__ __device__ static constexpr uint32_t T_OD(int g) { return T_O(g) + D; }
     static constexpr uint32_t T_S = ALT ? 4 * D : 2 * D;
@@ -131,7 +144,7 @@ struct Cfg {
     // keys 16kk..16kk+15 inside an S buffer
     __host__ __device__ static constexpr uint32_t t_pk(int kk, bool pd)
     {
-        return ALT ? (pd ? 32 : 0) + kk * 8 : BN + (kk >> 1) * 32 + (pd ? 16 : 0) + (kk & 1) * 8;
+        return BN + (kk >> 1) * 32 + (pd ? 16 : 0) + (kk & 1) * 8;
     }
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, 2 * BN, false);
     static constexpr uint32_t IDESC_SD = idesc_bf16_f32(BM, BN, false);
@@ -547,6 +560,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
     uint64_t *drain = pd_full + 2;
     uint64_t *s_full = drain + 1;        // by tiles: [2] S of warpgroup g's key tile written
     uint64_t *o_done = s_full + 2;       // by tiles: [2] PV of warpgroup g's key tile done
+    uint64_t *s_free = o_done + 2;       // by tiles: [2] warpgroup g has read its S buffer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -567,6 +581,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             if (C::ALT) {
                 mbar_init(&s_full[s], 1);
                 mbar_init(&o_done[s], 1);
+                mbar_init(&s_free[s], C::P_ARRIVALS);
             }
         }
         mbar_init(drain, 1);
@@ -728,6 +743,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         // operand is formed.  `first`: the first key tile of the query tile
         // for these accumulators, which starts them.  By tiles, key tile gg
         // goes into warpgroup (gg % 2)'s O_g and O'_g.
+        // By tiles the A operand (P or P (sS' - c), 64 keys = one 128-byte
+        // swizzle row per query row) comes from warpgroup ow's shared slot;
+        // by columns from TMEM, over S'_raw.
         auto issue_pa = [&](const int gk, const bool first) {
             const int s = gk % C::NV;
             tc_fence_after();
@@ -735,10 +753,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const int ow = C::ALT ? (gk & 1) : 0;
             const uint64_t dv = sdesc_sw128(smem_addr(smem + C::OFF_V + s * C::VST_BYTES), LBO, 1024);
             static_assert(C::VHALF_BYTES == C::NKB * LBO, "V' blocks follow V's at the block stride");
+            const uint64_t dp = sdesc_sw128(smem_addr(smem + C::off_p(ow, false)), 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)  // [O | O'_acc] += P [V | V']  (with V' = 0: O += P V)
-                mma_ts(tbase + C::T_O(ow), tP + C::t_pk(kk, false), desc_add(dv, kk * 2048),
-                       ZKV ? C::IDESC_PV : C::IDESC_PVV, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BN / 16; ++kk) {  // [O | O'_acc] += P [V | V']  (with V' = 0: O += P V)
+                if constexpr (C::ALT)
+                    mma_ss(tbase + C::T_O(ow), desc_add(dp, kk * 32), desc_add(dv, kk * 2048),
+                           ZKV ? C::IDESC_PV : C::IDESC_PVV, (!first || kk > 0) ? 1u : 0u);
+                else
+                    mma_ts(tbase + C::T_O(ow), tP + C::t_pk(kk, false), desc_add(dv, kk * 2048),
+                           ZKV ? C::IDESC_PV : C::IDESC_PVV, (!first || kk > 0) ? 1u : 0u);
+            }
         };
         auto issue_pb = [&](const int gk, const bool first) {
             const int s = gk % C::NV;
@@ -746,10 +770,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const uint32_t tP = tbase + C::T_S + (gk & 1) * (2 * BN);
             const int ow = C::ALT ? (gk & 1) : 0;
             const uint64_t dv = sdesc_sw128(smem_addr(smem + C::OFF_V + s * C::VST_BYTES), LBO, 1024);
+            const uint64_t dp = sdesc_sw128(smem_addr(smem + C::off_p(ow, true)), 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)  // O'_acc += P(sS' - c) V (with V' = 0 it starts O'_acc)
-                mma_ts(tbase + C::T_OD(ow), tP + C::t_pk(kk, true), desc_add(dv, kk * 2048), C::IDESC_PV,
-                       (!ZKV || !first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BN / 16; ++kk) {  // O'_acc += P(sS' - c) V (with V' = 0 it starts O'_acc)
+                if constexpr (C::ALT)
+                    mma_ss(tbase + C::T_OD(ow), desc_add(dp, kk * 32), desc_add(dv, kk * 2048), C::IDESC_PV,
+                           (!ZKV || !first || kk > 0) ? 1u : 0u);
+                else
+                    mma_ts(tbase + C::T_OD(ow), tP + C::t_pk(kk, true), desc_add(dv, kk * 2048), C::IDESC_PV,
+                           (!ZKV || !first || kk > 0) ? 1u : 0u);
+            }
             mma_commit(&vo_done[s]);
             if (C::ALT) mma_commit(&o_done[ow]);
         };
@@ -763,7 +793,47 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         bool ok = true;
         int lc = 0, gg = 0;
         Tile t;
-        for (int k = 0; ok; ++k) {
+        // By tiles: per query tile S_0 and S_1 first; then for key tile j,
+        // P V_j, S_{j+2} as soon as warpgroup (j % 2) has read S_j and S'_j
+        // from its buffer, and P (sS' - c) V_j.  S_{j+2} thus runs on the
+        // tensor core while that warpgroup's softmax still works on key tile j.
+        for (int k = 0; C::ALT && ok; ++k) {
+            const int it = item_of(p, k, t);
+            if (it == ITEM_END) break;
+            if (it == ITEM_SKIP || t.nT == 0) continue;
+            ok = wait_u(q_full, lc & 1, SITE_Q_FULL);
+            ++lc;
+            for (int j = 0; ok && j < 2 && j < t.nT; ++j) {
+                ok = wait_u(&k_full[(gg + j) % C::NK], ((gg + j) / C::NK) & 1, SITE_K_FULL);
+                if (!ok) break;
+                issue_s(gg + j);
+                if (lane == 0) stamp(gg + j, EV_S_ISSUE);
+            }
+            if (!ok) break;
+            if (t.nT <= 2) mma_commit(q_empty);  // that was the tile's last S
+            for (int j = 0; j < t.nT; ++j) {
+                const int gk = gg + j;
+                if (j + 2 < t.nT) {
+                    ok = wait_u(&s_free[gk & 1], (gk >> 1) & 1, SITE_S_FREE);
+                    if (ok) ok = wait_u(&k_full[(gk + 2) % C::NK], ((gk + 2) / C::NK) & 1, SITE_K_FULL);
+                    if (!ok) break;
+                    issue_s(gk + 2);
+                    if (lane == 0) stamp(gk + 2, EV_S_ISSUE);
+                    if (j + 3 == t.nT) mma_commit(q_empty);
+                }
+                ok = wait_u(&v_full[gk % C::NV], (gk / C::NV) & 1, SITE_V_FULL);
+                if (ok) ok = wait_u(&p_full[gk & 1], (gk >> 1) & 1, SITE_P_FULL);
+                if (!ok) break;
+                issue_pa(gk, j < 2);
+                if (lane == 0) stamp(gk, EV_PA_ISSUE);
+                ok = wait_u(&pd_full[gk & 1], (gk >> 1) & 1, SITE_P_FULL);
+                if (!ok) break;
+                issue_pb(gk, j < 2);
+                if (lane == 0) stamp(gk, EV_PB_ISSUE);
+            }
+            gg += t.nT;
+        }
+        for (int k = 0; !C::ALT && ok; ++k) {
             const int it = item_of(p, k, t);
             if (it == ITEM_END) break;
             if (it == ITEM_SKIP || t.nT == 0) continue;
@@ -787,7 +857,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 ok = wait_u(&v_full[gk % C::NV], (gk / C::NV) & 1, SITE_V_FULL);
                 if (ok) ok = wait_u(&p_full[gk & 1], (gk >> 1) & 1, SITE_P_FULL);
                 if (!ok) break;
-                const bool first = C::ALT ? j < 2 : j == 0;
+                const bool first = j == 0;
                 issue_pa(gk, first);
                 if (lane == 0) stamp(gk, EV_PA_ISSUE);
                 ok = wait_u(&pd_full[gk & 1], (gk >> 1) & 1, SITE_P_FULL);
@@ -827,10 +897,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 if (itk == ITEM_END) break;
                 if (itk == ITEM_SKIP) continue;
                 const int grow = t.q0 + r;
-                __nv_bfloat16 *out_ptr =
-                    static_cast<__nv_bfloat16 *>(g == 0 ? p.o : p.od) + (static_cast<size_t>(t.bh) * p.Lq + grow) * D;
-                const size_t lrow = static_cast<size_t>(t.bh) * p.Lq + grow;
+                // output row pointers, formed where they are used so they need
+                // no registers across the key loop
+                auto out_row = [&]() {
+                    return static_cast<__nv_bfloat16 *>(g == 0 ? p.o : p.od) +
+                           (static_cast<size_t>(t.bh) * p.Lq + grow) * D;
+                };
+                auto lse_row = [&]() { return static_cast<size_t>(t.bh) * p.Lq + grow; };
                 if (t.nT == 0) {
+                    __nv_bfloat16 *out_ptr = out_row();
+                    const size_t lrow = lse_row();
                     if (grow < p.Lq) {
                         const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
@@ -856,21 +932,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     tc_fence_after();
                     const int vt = nb - (t.jb + j) * BN;  // valid keys in the tile
                     const bool tail = vt < BN;
-                    uint32_t ra[32], rb[32];
+                    uint32_t ra[32], rb[32], rd[32];
                     tmem_ld32(tS, ra);       // S, keys 0..31
                     tmem_ld32(tS + 32, rb);  // S, keys 32..63
+                    tmem_ld32(tS + BN, rd);  // S'_raw, keys 0..31
                     tmem_ld_wait2(ra, rb);
+                    tmem_ld_ready(rd);
                     if (tail) {
+                        // padded keys: S to the pad (p = 0 below), S'_raw to 0 so
+                        // that P (sS' - c) = 0 (-c) = 0 whatever their bits were
                         const float pad = neg ? INFINITY : -INFINITY;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
                             ra[i] = (i < vt) ? ra[i] : f2u(pad);
                             rb[i] = (i + 32 < vt) ? rb[i] : f2u(pad);
+                            rd[i] = (i < vt) ? rd[i] : 0u;
                         }
                     }
                     const float mx = neg ? row_min64(ra, rb) : row_max64(ra, rb);
-                    uint32_t rd[32];
-                    tmem_ld32(tS + BN, rd);  // S'_raw, keys 0..31 (waited for below)
                     const float m_tile = mx * sl2;
                     float alpha = 1.f;
                     bool rescale = false;
@@ -883,8 +962,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                     l *= alpha;
                     acc_a *= alpha;
-                    float x[64];
+                    uint32_t pk[32];  // bf16 P, keys 2i and 2i + 1 (low half: key 2i)
                     {
+                        float x[64];
                         const uint64_t sl22 = f2_pack(sl2, sl2);
                         const uint64_t nm2 = f2_pack(-m_used, -m_used);
 #pragma unroll
@@ -892,31 +972,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                             float t0, t1, t2, t3;
                             f2_unpack(f2_fma(f2_pack(u2f(ra[2 * i]), u2f(ra[2 * i + 1])), sl22, nm2), t0, t1);
                             f2_unpack(f2_fma(f2_pack(u2f(rb[2 * i]), u2f(rb[2 * i + 1])), sl22, nm2), t2, t3);
-                            // pairs (i, a) and (i, b): quarter q of the 4 values goes to the
-                            // FMA pipe when q < POLY_QUARTERS (b pairs first, odd i first)
-                            constexpr int PQ = C::POLY_QUARTERS;
-                            const bool poly_b = PQ >= 2 || (PQ == 1 && (i & 1));
-                            const bool poly_a = PQ >= 4 || (PQ == 3 && (i & 1));
-                            if (poly_a) {
-                                ex2_poly2(t0, t1, x[2 * i], x[2 * i + 1]);
-                            } else {
-                                x[2 * i] = ex2_approx(t0);
-                                x[2 * i + 1] = ex2_approx(t1);
-                            }
-                            if (poly_b) {
-                                ex2_poly2(t2, t3, x[32 + 2 * i], x[33 + 2 * i]);
-                            } else {
-                                x[32 + 2 * i] = ex2_approx(t2);
-                                x[33 + 2 * i] = ex2_approx(t3);
-                            }
+                            x[2 * i] = ex2_approx(t0);
+                            x[2 * i + 1] = ex2_approx(t1);
+                            x[32 + 2 * i] = ex2_approx(t2);
+                            x[33 + 2 * i] = ex2_approx(t3);
                         }
-                    }
-                    if (tail) {
-                        // padded keys: p = 0 exactly (the pad times a zero scale is NaN)
+                        if (tail) {
+                            // padded keys: p = 0 exactly (the pad times a zero scale is NaN)
 #pragma unroll
-                        for (int i = 0; i < 64; ++i) x[i] = (i < vt) ? x[i] : 0.f;
-                    }
-                    {
+                            for (int i = 0; i < 64; ++i) x[i] = (i < vt) ? x[i] : 0.f;
+                        }
                         uint64_t s0 = f2_pack(x[0], x[1]), s1 = f2_pack(x[2], x[3]);
                         uint64_t s2 = f2_pack(x[32], x[33]), s3 = f2_pack(x[34], x[35]);
 #pragma unroll
@@ -930,21 +995,58 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         f2_unpack(f2_add(s0, s2), u0, u1);
                         f2_unpack(f2_add(s1, s3), u2, u3);
                         l += (u0 + u1) + (u2 + u3);
-                    }
-                    // The PV MMAs of this warpgroup's previous key tile, which
-                    // write O_g, are done: they were issued before this tile's
-                    // S, and S's commit (seen above) arrives only when every
-                    // MMA issued before it is done.  O_g may be rescaled at once.
-                    if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-                        for (int c = 0; c < 2 * D; c += 32) {  // O_g then O'_g
-                            uint32_t tt[32];
-                            tmem_ld32(tbase + lane_off + C::T_O(g) + c, tt);
-                            tmem_ld_wait(tt);
+                        if (nown == 0) {
+                            // centring constant c: the p-weighted mean of s S' over
+                            // keys 0..31 of this warpgroup's first key tile.  Their
+                            // p can all be 0 (the tile's max among keys 32..63 and
+                            // keys 0..31 more than ~87 logits below it); c cancels
+                            // exactly, so any finite value is right, and 0 is taken.
+                            float n0 = 0.f, n1 = 0.f, w0 = 0.f, w1 = 0.f;
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) tt[i] = f2u(u2f(tt[i]) * alpha);
-                            tmem_st32(tbase + lane_off + C::T_O(g) + c, tt);
+                            for (int i = 0; i < 32; i += 2) {
+                                n0 += (tail && i >= vt) ? 0.f : x[i] * (u2f(rd[i]) * sc);
+                                n1 += (tail && i + 1 >= vt) ? 0.f : x[i + 1] * (u2f(rd[i + 1]) * sc);
+                                w0 += x[i];
+                                w1 += x[i + 1];
+                            }
+                            const float wsum = w0 + w1;
+                            cctr = wsum > 0.f ? (n0 + n1) / wsum : 0.f;
                         }
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+                    }
+                    // The rest of S'_raw; then the buffer has been read, and the
+                    // MMA warp may put this warpgroup's next S there.
+                    uint32_t re[32];
+                    tmem_ld32(tS + BN + 32, re);  // S'_raw, keys 32..63
+                    tmem_ld_wait(re);
+                    if (tail) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) re[i] = (i + 32 < vt) ? re[i] : 0u;
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s_free[g]);
+                    // This warpgroup's previous key tile (gk - 2, possibly of an
+                    // earlier query tile): its PV MMAs read the P slots and
+                    // write O_g, and must be done before either is touched.
+                    // S_gk was issued without waiting for them.
+                    if (gk >= 2 &&
+                        !__all_sync(0xffffffffu, wait_bar_fast(&o_done[g], ((gk - 2) >> 1) & 1, wc, SITE_O_DONE))) {
+                        err = true;
+                        break;
+                    }
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int c = 0; c < 2 * D; c += 16) {  // O_g then O'_g
+                            uint32_t tt[16];
+                            tmem_ld16_wait(tbase + lane_off + C::T_O(g) + c, tt);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) tt[i] = f2u(u2f(tt[i]) * alpha);
+                            tmem_st16(tbase + lane_off + C::T_O(g) + c, tt);
+                        }
+                        tmem_st_wait();
                     }
                     if (tail) {
                         // Zero the V (and V') rows of padded keys so their bits
@@ -963,67 +1065,52 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                             *reinterpret_cast<uint4 *>(vst + blk * (BN * 128) + (vt + (rem >> 3)) * 128 +
                                                        (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
                         }
-                        fence_proxy_async_smem();
                     }
-                    {
-                        uint32_t pk[32];
+                    // Row r of a P slot: 64 keys in 8 chunks of 16 bytes, chunk
+                    // c at position c ^ (r % 8) of the row (the 128-byte swizzle
+                    // the MMA descriptor names); 8 consecutive rows fill all
+                    // 32 banks, so a warp's store takes the minimum 4 wavefronts.
+                    const uint32_t prow = smem_addr(smem + C::off_p(g, false)) + (r >> 3) * 1024 + (r & 7) * 128;
+                    const uint32_t pdrow = prow + C::P_BYTES;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-                        tmem_st32(tS, pk);  // P over S columns [0, 32): S has been read
-                    }
-                    tmem_st_wait();
-                    tc_fence_before();
+                    for (int c = 0; c < 8; ++c)
+                        st_shared_v4(prow + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                    // the tensor core reads P (and zeroed V rows) through the async proxy
+                    fence_proxy_async_smem();
+                    tc_fence_before();  // orders the rescale's TMEM stores before the PV MMAs
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&p_full[g]);
                     if (tracer) stamp(gk, EV_SM_P + 3 * g);
-                    // ---- bf16 P (s S' - c) while the tensor core multiplies P
-                    tmem_ld_wait(rd);
-                    if (nown == 0) {
-                        // centring constant c: the p-weighted mean of s S' over
-                        // keys 0..31 of this warpgroup's first key tile.  Their
-                        // p can all be 0 (the tile's max among keys 32..63 and
-                        // keys 0..31 more than ~87 logits below it); c cancels
-                        // exactly, so any finite value is right, and 0 is taken.
-                        float n0 = 0.f, n1 = 0.f, w0 = 0.f, w1 = 0.f;
-#pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            n0 += (tail && i >= vt) ? 0.f : x[i] * (u2f(rd[i]) * sc);
-                            n1 += (tail && i + 1 >= vt) ? 0.f : x[i + 1] * (u2f(rd[i + 1]) * sc);
-                            w0 += x[i];
-                            w1 += x[i + 1];
-                        }
-                        const float wsum = w0 + w1;
-                        cctr = wsum > 0.f ? (n0 + n1) / wsum : 0.f;
-                    }
-                    uint32_t re[32];
-                    tmem_ld32(tS + BN + 32, re);  // S'_raw, keys 32..63
+                    // ---- bf16 P (s S' - c) while the tensor core multiplies P.  p
+                    // is taken as rounded to bf16, the same p the P V MMAs use
+                    // (the fp32 p would need 32 more registers here).
                     const uint64_t sc2 = f2_pack(sc, sc);
                     const uint64_t nc2 = f2_pack(-cctr, -cctr);
                     uint64_t a0 = 0, a1 = 0;
-                    // keys [32h, 32h + 32) from v (S'_raw) into TMEM column 32 + 16h
+                    // keys [32h, 32h + 32) from v (S'_raw): chunks 4h..4h+3 of the row
                     auto pd_half = [&](const uint32_t (&v)[32], const int h) {
-                        uint32_t pdk[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int k0 = 32 * h + 2 * i;
-                            const uint64_t p2 = f2_pack(x[k0], x[k0 + 1]);
-                            const uint64_t d2 = f2_mul(f2_fma(f2_pack(u2f(v[2 * i]), u2f(v[2 * i + 1])), sc2, nc2), p2);
-                            float d0, d1;
-                            f2_unpack(d2, d0, d1);
-                            if (tail) {
-                                d0 = (k0 < vt) ? d0 : 0.f;
-                                d1 = (k0 + 1 < vt) ? d1 : 0.f;
+                        for (int cc = 0; cc < 4; ++cc) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const int i = 4 * cc + q;
+                                const uint32_t pp = pk[16 * h + i];
+                                const uint64_t p2 = f2_pack(u2f(pp << 16), u2f(pp & 0xFFFF0000u));
+                                const uint64_t d2 =
+                                    f2_mul(f2_fma(f2_pack(u2f(v[2 * i]), u2f(v[2 * i + 1])), sc2, nc2), p2);
+                                float d0, d1;
+                                f2_unpack(d2, d0, d1);
+                                w[q] = pack_bf16x2(d0, d1);
+                                // the two rounded values as fp32
+                                const uint64_t r2 = f2_pack(u2f(w[q] << 16), u2f(w[q] & 0xFFFF0000u));
+                                if (i & 1) a1 = f2_add(a1, r2);
+                                else a0 = f2_add(a0, r2);
                             }
-                            pdk[i] = pack_bf16x2(d0, d1);
-                            // the two rounded values as fp32
-                            const uint64_t r2 = f2_pack(u2f(pdk[i] << 16), u2f(pdk[i] & 0xFFFF0000u));
-                            if (i & 1) a1 = f2_add(a1, r2);
-                            else a0 = f2_add(a0, r2);
+                            st_shared_v4(pdrow + (((4 * h + cc) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
                         }
-                        tmem_st16(tS + 32 + 16 * h, pdk);
                     };
                     pd_half(rd, 0);
-                    tmem_ld_wait(re);
                     pd_half(re, 1);
                     {
                         float u0, u1, u2, u3;
@@ -1031,8 +1118,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         f2_unpack(a1, u2, u3);
                         acc_a += (u0 + u1) + (u2 + u3);
                     }
-                    tmem_st_wait();
-                    tc_fence_before();
+                    fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pd_full[g]);
                     if (tracer) stamp(gk, EV_SM_PD + 3 * g);
@@ -1074,6 +1160,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 // m = M, l = L, c = mu, a = 0, O = sum_h b_h O_h and
                 // O' = sum_h b_h (O'_h + (c_h - mu) O_h).
                 const bool part = t.part >= 0;
+                __nv_bfloat16 *out_ptr = out_row();
+                const size_t lrow = lse_row();
                 const float wn = part ? 1.f : inv_l;
                 const float w0 = b0 * wn, w1 = b1 * wn;
                 const float k0 = w0 * (c0v - mu), k1 = w1 * (c1v - mu);
