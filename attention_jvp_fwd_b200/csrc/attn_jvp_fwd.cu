@@ -120,8 +120,8 @@ struct Cfg {
     __host__ __device__ static constexpr uint32_t off_p(int g, bool pd) { return OFF_P + (2 * g + (pd ? 1 : 0)) * P_BYTES; }
     static constexpr uint32_t OFF_BAR = OFF_P + (ALT ? 4 * P_BYTES : 0);
     // q_full, q_empty, k_full[NK], ks_done[NK], v_full[NV], vo_done[NV],
-    // p_full[2], pd_full[2], drain, and by tiles s_full[2], o_done[2], s_free[2]
-    static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 2 + 2 + 1 + (ALT ? 6 : 0);
+    // p_full[2], pd_full[2], drain, and by tiles s_free[2]
+    static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 2 + 2 + 1 + (ALT ? 2 : 0);
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem slot, abort flag
     // Softmax exchange, floats.  By columns: per-warpgroup partial l, a
     // ([2][2][128]) and the centring constant hand-off ([128]).  By tiles:
@@ -543,24 +543,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
     uint64_t *q_empty = q_full + 1;  // the last S MMA of a query tile has read Q, Q'
     uint64_t *k_full = q_empty + 1;
     // ks_done[s]: the S MMAs of the key tile in K slot s are done, so the slot
-    // may be refilled (and, by columns, the softmax may read S).  vo_done[s]:
+    // may be refilled (and the softmax may read S).  vo_done[s]:
     // the PV MMAs of the key tile in V slot s are done, so the slot may be
-    // refilled (and, by columns, O may be rescaled or read).  By columns one
-    // commit per MMA group thus signals both consumers; neither can fall two
-    // phases behind on a slot, because the next phase needs the slot's next
-    // load, issued by the TMA warp only after its wait, and the MMAs of a key
-    // tile that this softmax warp has not yet written P for.  By tiles the
-    // softmax keeps barriers of its own (s_full[g], o_done[g] for warpgroup
-    // g), which measured faster there.
+    // refilled (and O may be rescaled or read).  One commit per MMA group
+    // thus signals both consumers (each commit costs the tensor pipe about 30
+    // clocks).  Neither can fall two phases behind on a slot: the next phase
+    // needs the slot's next load, issued by the TMA warp only after its wait,
+    // and MMAs that the MMA warp issues, in a fixed order, only after P
+    // signals of key tiles that the waiting softmax warp has not yet reached.
     uint64_t *ks_done = k_full + C::NK;
     uint64_t *v_full = ks_done + C::NK;
     uint64_t *vo_done = v_full + C::NV;
     uint64_t *p_full = vo_done + C::NV;  // [2] bf16 P written
     uint64_t *pd_full = p_full + 2;      // [2] bf16 P (sS' - c) written
     uint64_t *drain = pd_full + 2;
-    uint64_t *s_full = drain + 1;        // by tiles: [2] S of warpgroup g's key tile written
-    uint64_t *o_done = s_full + 2;       // by tiles: [2] PV of warpgroup g's key tile done
-    uint64_t *s_free = o_done + 2;       // by tiles: [2] warpgroup g has read its S buffer
+    uint64_t *s_free = drain + 1;        // by tiles: [2] warpgroup g has read its S buffer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -578,11 +575,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         for (int s = 0; s < 2; ++s) {
             mbar_init(&p_full[s], C::P_ARRIVALS);
             mbar_init(&pd_full[s], C::P_ARRIVALS);
-            if (C::ALT) {
-                mbar_init(&s_full[s], 1);
-                mbar_init(&o_done[s], 1);
-                mbar_init(&s_free[s], C::P_ARRIVALS);
-            }
+            if (C::ALT) mbar_init(&s_free[s], C::P_ARRIVALS);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -732,7 +725,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 mma_ss(tS + BN, desc_add(dqd, oa), desc_add(dk, ob), C::IDESC_SD, (!ZKV || kk > 0) ? 1u : 0u);
             }
             mma_commit(&ks_done[s]);
-            if (C::ALT) mma_commit(&s_full[gk & 1]);
             issued = true;
         };
         // LBO: distance between 64-column blocks of V
@@ -781,7 +773,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                            (!ZKV || !first || kk > 0) ? 1u : 0u);
             }
             mma_commit(&vo_done[s]);
-            if (C::ALT) mma_commit(&o_done[ow]);
         };
         // Fixed order per query tile: S_0, S_1, PV_0, S_2, PV_1, ...: S_{j+1}
         // runs on the tensor core while the softmax works on key tile j, and
@@ -924,7 +915,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 int nown = 0, last = 0;
                 for (int j = ((gg & 1) == g) ? 0 : 1; j < nT; j += 2) {
                     const int gk = gg + j;
-                    if (!__all_sync(0xffffffffu, wait_bar_fast(&s_full[g], (gk >> 1) & 1, wc, SITE_S_FULL))) {
+                    if (!__all_sync(0xffffffffu, wait_bar_fast(&ks_done[gk % C::NK], (gk / C::NK) & 1, wc, SITE_S_FULL))) {
                         err = true;
                         break;
                     }
@@ -1031,8 +1022,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     // earlier query tile): its PV MMAs read the P slots and
                     // write O_g, and must be done before either is touched.
                     // S_gk was issued without waiting for them.
-                    if (gk >= 2 &&
-                        !__all_sync(0xffffffffu, wait_bar_fast(&o_done[g], ((gk - 2) >> 1) & 1, wc, SITE_O_DONE))) {
+                    if (gk >= 2 && !__all_sync(0xffffffffu, wait_bar_fast(&vo_done[(gk - 2) % C::NV],
+                                                                          ((gk - 2) / C::NV) & 1, wc, SITE_O_DONE))) {
                         err = true;
                         break;
                     }
@@ -1128,7 +1119,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 bool ok;
                 {
                     bool done = !err;
-                    if (!err && nown > 0) done = wait_bar(&o_done[g], (last >> 1) & 1, wc, SITE_O_DONE, true);
+                    if (!err && nown > 0)
+                        done = wait_bar(&vo_done[last % C::NV], (last / C::NV) & 1, wc, SITE_O_DONE, true);
                     ok = bar_and(BAR_SOFT, NSOFT, done);  // reached by all 256 threads
                 }
                 // whether warpgroup h had key tiles in this query tile (the same
