@@ -181,3 +181,37 @@ def test_centring_window_underflow(d, masked):
     assert bool(torch.all(torch.isfinite(o.float()))) and bool(torch.all(torch.isfinite(od.float())))
     assert bool(torch.all(torch.isfinite(lse)))
     compare(gpu_rows(o, od, lse), oracle_ref(w, scale=1.0), f"centring underflow d{d} masked={masked}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("split", [
+    pytest.param(False, marks=pytest.mark.xfail(
+        strict=True,
+        reason="known limit: the centring constant comes from a query tile's first key tile; with sS' "
+               "drifting by about 40 along the keys the bf16 P (sS' - c) of the dominant keys carry "
+               "rounding about 40 * 2^-9, and O' misses the 2e-2 bar (6.1e-2 at d = 64, 8.1e-2 at d = 128)")),
+    True])
+def test_rescale_every_key_tile(d, split):
+    """Logits and tangent logits that grow along the key axis (0.1 per key
+    at scale 1, about 9 log2 units per 64-key tile): the row max passes the
+    lazy-rescale threshold (2^4) in every key tile, so O and O'_acc are
+    rescaled every tile, each time after the previous tile's PV MMAs are
+    done.  With the split, the 4 query tiles are cut into key ranges with a
+    centring constant each, merged at the end: within the bar.  Without it,
+    each query tile walks all 7 key tiles (a ragged last one of 17 keys) with
+    the first tile's centring constant, and O' misses the bar."""
+    from attention_jvp_fwd_b200 import api, attn_jvp_fwd
+    B, H, Lq, Lk = 1, 2, 200, 6 * 64 + 17
+    w = W.make_custom(B, H, Lq, Lk, d, seed=77)
+    q = 0.1 * W.bf16_bits_to_f32(w.q)
+    k = 0.1 * W.bf16_bits_to_f32(w.k)
+    q[..., 0] = 1.0
+    k[..., :, 0] = 0.1 * np.arange(Lk, dtype=np.float32)
+    w.q = W.bf16_round_bits(q)
+    w.k = W.bf16_round_bits(k)
+    ins = [to_dev(x) for x in w.inputs()]
+    o, od, lse = attn_jvp_fwd(*ins, scale=1.0, split=split)
+    torch.cuda.synchronize()
+    st, site = api.attn_jvp_check()
+    assert st == 0, f"device status {st} at site {site}"
+    compare(gpu_rows(o, od, lse), oracle_ref(w, scale=1.0), f"rescale every tile d{d} split={split}")
